@@ -1,0 +1,117 @@
+"""Planted mistakes in the oracle must be caught by its pins.
+
+Each mutant is a one-line change to a copy of the oracle's source, made here
+on the CPU (the oracle on disk is untouched). The pin tests of
+test_oracle_attention.py / test_oracle_unmask.py are then run against the
+mutated copy; at least one of them has to fail, or the pins would not protect
+against that kind of mistake (a dropped term, a wrong sign or index, a wrong
+operand, an off-by-one).
+"""
+
+import importlib.util
+import inspect
+import os
+
+import pytest
+
+import test_oracle_attention as TA
+import test_oracle_unmask as TU
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _load_mutant(relpath, old, new, name):
+    src = open(os.path.join(ROOT, relpath)).read()
+    assert src.count(old) >= 1, f"mutation site not found: {old!r}"
+    src = src.replace(old, new)
+    spec = importlib.util.spec_from_loader(name, loader=None)
+    mod = importlib.util.module_from_spec(spec)
+    exec(compile(src, f"<mutant {name}>", "exec"), mod.__dict__)
+    return mod
+
+
+def _collect(module):
+    """All pin tests of a module as (callable, list-of-arg-dicts)."""
+    out = []
+    for nm, fn in inspect.getmembers(module, inspect.isfunction):
+        if not nm.startswith("test_"):
+            continue
+        marks = getattr(fn, "pytestmark", [])
+        params = [m for m in marks if m.name == "parametrize"]
+        if params:
+            argnames = params[0].args[0]
+            values = params[0].args[1]
+            names = [a.strip() for a in argnames.split(",")]
+            calls = []
+            for v in values:
+                v = v if len(names) > 1 else (v,)
+                calls.append(dict(zip(names, v)))
+            out.append((fn, calls))
+        else:
+            out.append((fn, [{}]))
+    return out
+
+
+def _some_pin_fails(module, patches, monkeypatch):
+    for attr, val in patches.items():
+        monkeypatch.setattr(module, attr, val)
+    for fn, calls in _collect(module):
+        for kw in calls:
+            try:
+                fn(**kw)
+            except Exception:
+                return True
+    return False
+
+
+ATTN_MUTANTS = [
+    ("scale 1/d", "scale = 1.0 / np.sqrt(d)", "scale = 1.0 / d"),
+    ("interleaved GQA", "    return h // g\n", "    return h % H_kv\n"),
+    ("block keys causal", "k_blk[b, :, kv, :]], axis=0)", "k_blk[b, :1, kv, :]], axis=0)"),
+    ("drop prefix", "[k_prefix[off:off + L, kv, :], k_blk", "[k_prefix[off:off, kv, :], k_blk"),
+    ("prefix off by one", "k_prefix[off:off + L, kv, :], k_blk[b, :, kv, :]",
+     "k_prefix[off + 1:off + L + 1, kv, :], k_blk[b, :, kv, :]"),
+    ("no normalisation", "o = (p @ V) / l", "o = (p @ V)"),
+    ("lse without max", "lse = mx[:, 0] + np.log(l[:, 0])", "lse = np.log(l[:, 0])"),
+    ("combine weights sign", "w = np.exp(lse_parts - M[None, :])", "w = np.exp(M[None, :] - lse_parts)"),
+]
+
+
+@pytest.mark.parametrize("mut", ATTN_MUTANTS, ids=[m[0] for m in ATTN_MUTANTS])
+def test_attention_mutant_is_caught(mut, monkeypatch):
+    name, old, new = mut
+    mod = _load_mutant("oracle/attention.py", old, new, "mut_attn")
+    patches = {"block_attention": mod.block_attention, "attend": mod.attend,
+               "lse_combine": mod.lse_combine, "block_attention_rows": mod.block_attention_rows}
+    assert _some_pin_fails(TA, patches, monkeypatch), f"no pin caught mutant {name!r}"
+
+
+UNMASK_MUTANTS = [
+    ("ties to highest id", "tok = int(np.flatnonzero(row == mx)[0])", "tok = int(np.flatnonzero(row == mx)[-1])"),
+    (">= instead of >", "commit[r] = conf[r] > thr", "commit[r] = conf[r] >= thr"),
+    ("no max shift in Z", "z = np.exp(row - mx).sum()", "z = np.exp(row).sum()"),
+    ("fallback ties to last", "best = masked[int(np.flatnonzero(c == c.max())[0])]",
+     "best = masked[int(np.flatnonzero(c == c.max())[-1])]"),
+    ("fallback picks min", "c == c.max()", "c == c.min()"),
+    ("mask not updated", '"mask_out": m & ~commit', '"mask_out": m'),
+    ("unmasked rows scored", "        if not m[r]:\n            continue\n", ""),
+]
+
+
+@pytest.mark.parametrize("mut", UNMASK_MUTANTS, ids=[m[0] for m in UNMASK_MUTANTS])
+def test_unmask_mutant_is_caught(mut, monkeypatch):
+    name, old, new = mut
+    mod = _load_mutant("oracle/unmask.py", old, new, "mut_unmask")
+    patches = {"confidence_unmask": mod.confidence_unmask, "top2_gap": mod.top2_gap}
+    assert _some_pin_fails(TU, patches, monkeypatch), f"no pin caught mutant {name!r}"
+
+
+def test_unmutated_copy_passes_every_pin(monkeypatch):
+    """Control: the loader itself does not make pins fail."""
+    mod = _load_mutant("oracle/attention.py", "import numpy as np", "import numpy as np", "same_attn")
+    patches = {"block_attention": mod.block_attention, "attend": mod.attend,
+               "lse_combine": mod.lse_combine, "block_attention_rows": mod.block_attention_rows}
+    assert not _some_pin_fails(TA, patches, monkeypatch)
+    mod = _load_mutant("oracle/unmask.py", "import numpy as np", "import numpy as np", "same_unmask")
+    assert not _some_pin_fails(TU, {"confidence_unmask": mod.confidence_unmask,
+                                    "top2_gap": mod.top2_gap}, monkeypatch)
