@@ -1,0 +1,194 @@
+"""Thin ctypes binding of libbd.so (include/bd.h).
+
+Argument marshalling only: shapes are read off the tensors, outputs and
+workspaces are allocated with torch when the caller does not pass them, and
+every computation runs in the library's CUDA kernels. There is no CPU
+fallback: if libbd.so is missing or cannot be loaded, the first call raises.
+"""
+
+import ctypes
+import os
+
+import torch
+
+_HERE = os.path.dirname(os.path.abspath(__file__))
+_LIB = None
+
+BD_OK = 0
+_DTYPES = {torch.float32: 0, torch.bfloat16: 1}
+
+
+class BdError(RuntimeError):
+    def __init__(self, status, where):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} ({status})")
+
+
+def lib_path():
+    return os.environ.get("BD_LIB", os.path.join(_HERE, "libbd.so"))
+
+
+def _lib():
+    global _LIB
+    if _LIB is not None:
+        return _LIB
+    path = lib_path()
+    if not os.path.exists(path):
+        raise RuntimeError(
+            f"libbd.so not found at {path}: build it first "
+            "(python -m block_diffusion_lm_bd_b200.build)")
+    lib = ctypes.CDLL(path)
+    c = ctypes
+    vp, i32, i64, f32, sz = c.c_void_p, c.c_int, c.c_int64, c.c_float, c.c_size_t
+    lib.bd_version.restype = i32
+    lib.bd_status_string.restype = c.c_char_p
+    lib.bd_status_string.argtypes = [i32]
+    lib.bd_launch_count.restype = c.c_uint64
+    lib.bd_attn_workspace_bytes.restype = sz
+    lib.bd_attn_workspace_bytes.argtypes = [i32] * 5
+    lib.bd_attn_step.restype = i32
+    lib.bd_attn_step.argtypes = [vp, vp, vp, i64, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32,
+                                 i32, vp, vp, vp, sz, vp]
+    lib.bd_unmask_workspace_bytes.restype = sz
+    lib.bd_unmask_workspace_bytes.argtypes = [i32, i32]
+    lib.bd_unmask.restype = i32
+    lib.bd_unmask.argtypes = [vp, vp, f32, vp, vp, vp, vp, i32, i32, i32, i32, vp, sz, vp]
+    lib.bd_get_device_status.restype = i32
+    lib.bd_get_device_status.argtypes = [vp]
+    lib.bd_debug_wait_timeout.restype = i32
+    lib.bd_debug_wait_timeout.argtypes = [i32, vp]
+    _LIB = lib
+    return lib
+
+
+def status_string(status):
+    return _lib().bd_status_string(int(status)).decode()
+
+
+def _check(status, where):
+    if status != BD_OK:
+        raise BdError(status, where)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+def _stream_ptr(stream, device):
+    if stream is None:
+        stream = torch.cuda.current_stream(device)
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _need(t, name, dtype=None, device=None):
+    if not isinstance(t, torch.Tensor) or not t.is_cuda:
+        raise ValueError(f"{name} must be a CUDA tensor")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+    if dtype is not None and t.dtype != dtype:
+        raise ValueError(f"{name} must be {dtype}, got {t.dtype}")
+    if device is not None and t.device != device:
+        raise ValueError(f"{name} is on {t.device}, expected {device}")
+
+
+def launch_count():
+    """Kernels launched through libbd so far in this process."""
+    return int(_lib().bd_launch_count())
+
+
+def attn_workspace_bytes(B, S, H_q, H_kv, d):
+    return int(_lib().bd_attn_workspace_bytes(B, S, H_q, H_kv, d))
+
+
+def unmask_workspace_bytes(rows, V):
+    return int(_lib().bd_unmask_workspace_bytes(rows, V))
+
+
+def attn_step(q, k_prefix, v_prefix, k_blk, v_blk, prefix_len, prefix_offset, scale=None,
+              o=None, lse=None, want_lse=True, workspace=None, stream=None):
+    """bd_attn_step on torch tensors. Returns (o float32 [B,S,H_q,d], lse or None)."""
+    B, S, H_q, d = q.shape
+    H_kv = k_blk.shape[2]
+    dev = q.device
+    if q.dtype not in _DTYPES:
+        raise ValueError(f"unsupported dtype {q.dtype}")
+    for t, nm in ((q, "q"), (k_prefix, "k_prefix"), (v_prefix, "v_prefix"), (k_blk, "k_blk"),
+                  (v_blk, "v_blk")):
+        _need(t, nm, q.dtype, dev)
+    _need(prefix_len, "prefix_len", torch.int32, dev)
+    _need(prefix_offset, "prefix_offset", torch.int64, dev)
+    if k_prefix.shape[1:] != (H_kv, d) or v_prefix.shape != k_prefix.shape:
+        raise ValueError("k_prefix / v_prefix must be [rows, H_kv, d]")
+    if k_blk.shape != (B, S, H_kv, d) or v_blk.shape != k_blk.shape:
+        raise ValueError("k_blk / v_blk must be [B, S, H_kv, d]")
+    if o is None:
+        o = torch.empty((B, S, H_q, d), dtype=torch.float32, device=dev)
+    _need(o, "o", torch.float32, dev)
+    if lse is None and want_lse:
+        lse = torch.empty((B, H_q, S), dtype=torch.float32, device=dev)
+    if lse is not None:
+        _need(lse, "lse", torch.float32, dev)
+    if workspace is None:
+        nbytes = attn_workspace_bytes(B, S, H_q, H_kv, d)
+        if nbytes == 0:
+            raise BdError(1, "bd_attn_workspace_bytes")
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    st = _lib().bd_attn_step(
+        _ptr(q), _ptr(k_prefix), _ptr(v_prefix), int(k_prefix.shape[0]), _ptr(k_blk),
+        _ptr(v_blk), _ptr(prefix_len), _ptr(prefix_offset), B, S, H_q, H_kv, d,
+        float(scale) if scale is not None else 0.0, _DTYPES[q.dtype], _ptr(o), _ptr(lse),
+        _ptr(workspace), workspace.numel() * workspace.element_size(),
+        _stream_ptr(stream, dev))
+    _check(st, "bd_attn_step")
+    return o, lse
+
+
+def unmask(logits, mask, gamma, block_S=0, commit_at_least_one=False, tokens_out=None,
+           conf_out=None, commit_out=None, mask_out=None, workspace=None, stream=None):
+    """bd_unmask on torch tensors.
+
+    mask_out: None (not written), a uint8 tensor, or "inplace" (update mask).
+    Returns dict(tokens, conf, commit, mask_out).
+    """
+    rows, V = logits.shape
+    dev = logits.device
+    _need(logits, "logits", torch.float32)
+    _need(mask, "mask", torch.uint8, dev)
+    if tokens_out is None:
+        tokens_out = torch.full((rows,), -1, dtype=torch.int32, device=dev)
+    if conf_out is None:
+        conf_out = torch.full((rows,), float("nan"), dtype=torch.float32, device=dev)
+    if commit_out is None:
+        commit_out = torch.empty((rows,), dtype=torch.uint8, device=dev)
+    if isinstance(mask_out, str) and mask_out == "inplace":
+        mask_out = mask
+    for t, nm, dt in ((tokens_out, "tokens_out", torch.int32), (conf_out, "conf_out", torch.float32),
+                      (commit_out, "commit_out", torch.uint8)):
+        _need(t, nm, dt, dev)
+    if mask_out is not None:
+        _need(mask_out, "mask_out", torch.uint8, dev)
+    if workspace is None:
+        nbytes = unmask_workspace_bytes(rows, V)
+        if nbytes == 0:
+            raise BdError(1, "bd_unmask_workspace_bytes")
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    st = _lib().bd_unmask(
+        _ptr(logits), _ptr(mask), float(gamma), _ptr(tokens_out), _ptr(conf_out),
+        _ptr(commit_out), _ptr(mask_out), rows, V, int(block_S), 1 if commit_at_least_one else 0,
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _stream_ptr(stream, dev))
+    _check(st, "bd_unmask")
+    return {"tokens": tokens_out, "conf": conf_out, "commit": commit_out, "mask_out": mask_out}
+
+
+def get_device_status(stream=None, device=None):
+    """Synchronise the stream; return (and clear) the device status code."""
+    if device is None:
+        device = torch.device("cuda", torch.cuda.current_device())
+    return int(_lib().bd_get_device_status(_stream_ptr(stream, device)))
+
+
+def debug_wait_timeout(max_polls, stream=None, device=None):
+    if device is None:
+        device = torch.device("cuda", torch.cuda.current_device())
+    _check(_lib().bd_debug_wait_timeout(int(max_polls), _stream_ptr(stream, device)),
+           "bd_debug_wait_timeout")

@@ -1,0 +1,162 @@
+// Attention of the active block over prefix ++ block keys: parameters,
+// workspace layout and the work plan shared by every attention kernel.
+//
+// Work units. For sequence b with L_b prefix rows, each KV head kv has
+// n_b = ceil(L_b / kUnitKeys) + 1 units: the prefix tiles of kUnitKeys keys
+// and, last, the block tile (the S keys of the active block). Units are
+// ordered (b, kv, unit) and the whole list of W = H_kv * sum_b n_b units is
+// split into G equal contiguous ranges, one per persistent CTA (G = SM
+// count). A CTA walks its range; each maximal run of units of one (b, kv)
+// pair is a segment, whose result is either final (the pair lies wholly in
+// the range: o and lse are written directly) or partial (written to one of
+// the CTA's two boundary slots and merged by attn_combine_kernel with the
+// log-sum-exp identity).
+//
+// Each CTA computes its own starting point with a block-wide scan of n_b
+// (no separate planning launch); CTA 0 also stores the scan for the combine.
+#pragma once
+
+#include "bd_common.cuh"
+
+namespace bd {
+
+constexpr int kUnitKeys = 128;     // prefix keys per work unit
+constexpr int kMaxBatch = 4096;    // sequences per call
+constexpr int kMaxRows = 128;      // packed query rows g*S per (b, kv)
+constexpr int kPlanThreads = 256;  // scan width of the in-kernel plan
+
+struct AttnWs {
+  int *flag;     // [1]  1: device-side argument error, nothing was written
+  int *cum;      // [B+1] exclusive scan of n_b
+  float *slot;   // [G][2][M][d]  partial outputs (normalised)
+  float *slot_lse;  // [G][2][M] partial log-sum-exp (natural log)
+};
+
+__host__ __device__ inline size_t attn_align(size_t x) { return (x + 255) & ~size_t(255); }
+
+__host__ __device__ inline size_t attn_ws_layout(int B, int M, int d, int G, AttnWs *ws,
+                                                 char *base) {
+  size_t off = 0;
+  if (ws) ws->flag = reinterpret_cast<int *>(base + off);
+  off = attn_align(off + sizeof(int));
+  if (ws) ws->cum = reinterpret_cast<int *>(base + off);
+  off = attn_align(off + sizeof(int) * size_t(B + 1));
+  if (ws) ws->slot = reinterpret_cast<float *>(base + off);
+  off = attn_align(off + sizeof(float) * size_t(G) * 2 * M * d);
+  if (ws) ws->slot_lse = reinterpret_cast<float *>(base + off);
+  off = attn_align(off + sizeof(float) * size_t(G) * 2 * M);
+  return off;
+}
+
+struct AttnParams {
+  const void *q;
+  const void *k_prefix;
+  const void *v_prefix;
+  const void *k_blk;
+  const void *v_blk;
+  const int32_t *prefix_len;
+  const int64_t *prefix_offset;
+  int64_t prefix_rows;
+  int B, S, H_q, H_kv, d, g, M;
+  float scale_log2;  // score scale * log2(e)
+  float *o;
+  float *lse;
+  AttnWs ws;
+  int G;
+  uint32_t max_polls;
+};
+
+__device__ __forceinline__ int attn_units(int L) { return (L + kUnitKeys - 1) / kUnitKeys + 1; }
+
+// Where a CTA's range starts, and the total work.
+struct PlanStart {
+  int64_t W;    // total units
+  int b;        // sequence of the first unit
+  int cum_b;    // sum of n over sequences before b
+  bool bad;     // some prefix_len / prefix_offset is out of range
+};
+
+// Block-wide plan: every thread of the CTA must call it. `e0` is the CTA's
+// first unit, computed from W inside (so passed as the CTA index).
+__device__ inline PlanStart attn_plan(const AttnParams &p, int cta, int *s_scan, int *s_misc) {
+  const int tid = threadIdx.x;
+  // pass 1: total units and range check
+  int carry = 0;
+  int bad = 0;
+  for (int base = 0; base < p.B; base += kPlanThreads) {
+    const int b = base + tid;
+    int n = 0;
+    if (b < p.B && tid < kPlanThreads) {
+      const int L = p.prefix_len[b];
+      const int64_t off = p.prefix_offset[b];
+      if (L < 0 || off < 0 || off + L > p.prefix_rows) bad = 1;
+      n = attn_units(L < 0 ? 0 : L);
+    }
+    if (tid < kPlanThreads) s_scan[tid] = n;
+    __syncthreads();
+    for (int o = 1; o < kPlanThreads; o <<= 1) {
+      int v = (tid < kPlanThreads && tid >= o) ? s_scan[tid - o] : 0;
+      __syncthreads();
+      if (tid < kPlanThreads) s_scan[tid] += v;
+      __syncthreads();
+    }
+    if (cta == 0 && b < p.B && tid < kPlanThreads) p.ws.cum[b] = carry + s_scan[tid] - n;
+    carry += s_scan[kPlanThreads - 1];
+    __syncthreads();
+  }
+  if (tid == 0) s_misc[0] = 0;
+  __syncthreads();
+  if (bad) atomicOr(&s_misc[0], 1);
+  __syncthreads();
+  PlanStart ps;
+  ps.bad = s_misc[0] != 0;
+  ps.W = int64_t(p.H_kv) * carry;
+  if (cta == 0 && tid == 0) {
+    p.ws.cum[p.B] = carry;
+    *p.ws.flag = ps.bad ? 1 : 0;
+  }
+  ps.b = 0;
+  ps.cum_b = 0;
+  if (ps.bad || ps.W == 0) return ps;
+  // pass 2: the sequence holding unit e0 = start(cta)
+  const int64_t e0 = part_start(cta, ps.W, p.G);
+  if (tid == 0) {
+    s_misc[1] = -1;
+    s_misc[2] = 0;
+  }
+  carry = 0;
+  __syncthreads();
+  for (int base = 0; base < p.B; base += kPlanThreads) {
+    const int b = base + tid;
+    int n = 0;
+    if (b < p.B && tid < kPlanThreads) n = attn_units(max(0, p.prefix_len[b]));
+    if (tid < kPlanThreads) s_scan[tid] = n;
+    __syncthreads();
+    for (int o = 1; o < kPlanThreads; o <<= 1) {
+      int v = (tid < kPlanThreads && tid >= o) ? s_scan[tid - o] : 0;
+      __syncthreads();
+      if (tid < kPlanThreads) s_scan[tid] += v;
+      __syncthreads();
+    }
+    if (b < p.B && tid < kPlanThreads) {
+      const int ex = carry + s_scan[tid] - n;
+      if (int64_t(p.H_kv) * ex <= e0 && e0 < int64_t(p.H_kv) * (ex + n)) {
+        s_misc[1] = b;
+        s_misc[2] = ex;
+      }
+    }
+    carry += s_scan[kPlanThreads - 1];
+    __syncthreads();
+  }
+  ps.b = s_misc[1];
+  ps.cum_b = s_misc[2];
+  __syncthreads();
+  return ps;
+}
+
+// Index of the boundary slot a segment writes to.
+__device__ __forceinline__ int64_t attn_slot_index(int cta, bool first) {
+  return 2 * int64_t(cta) + (first ? 0 : 1);
+}
+
+}  // namespace bd

@@ -1,0 +1,233 @@
+// Split-KV attention of the active block on the CUDA cores (fp32 FFMA).
+//
+// This is the fp32 path (inputs stored as float32, where tensor-core tf32
+// would not meet a 1e-4 tolerance) and a portable path for bf16 inputs. Each
+// persistent CTA walks its range of work units (attn_common.cuh); per segment
+// it stages the g*S packed queries of one (b, kv) pair in shared memory and
+// streams the pair's keys 32 at a time: scores (lane = key), an online
+// softmax in base 2 per row (a warp owns rows warp + 8 i), and P.V with each
+// lane owning 4 output columns.
+#pragma once
+
+#include "attn_common.cuh"
+
+namespace bd {
+
+constexpr int kSimtThreads = 256;
+constexpr int kSimtKeys = 32;
+
+template <int D>
+__host__ __device__ constexpr size_t simt_smem_bytes() {
+  return sizeof(float) * (size_t(kMaxRows) * D + kSimtKeys * (D + 4) + kSimtKeys * D +
+                          kMaxRows * (kSimtKeys + 1) + 2 * kMaxRows);
+}
+
+template <typename T, int D>
+__global__ void __launch_bounds__(kSimtThreads, 1) attn_simt_kernel(AttnParams p) {
+  extern __shared__ __align__(16) float smem[];
+  float *Qs = smem;                              // [kMaxRows][D]
+  float *Ks = Qs + kMaxRows * D;                 // [32][D+4]
+  float *Vs = Ks + kSimtKeys * (D + 4);          // [32][D]
+  float *Ps = Vs + kSimtKeys * D;                // [kMaxRows][33]
+  float *s_alpha = Ps + kMaxRows * (kSimtKeys + 1);  // [kMaxRows]
+  float *s_l = s_alpha + kMaxRows;               // [kMaxRows]
+  __shared__ int s_scan[kPlanThreads];
+  __shared__ int s_misc[4];
+
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int cta = blockIdx.x;
+  const PlanStart ps = attn_plan(p, cta, s_scan, s_misc);
+  pdl_launch_dependents();
+  if (ps.bad) {
+    if (cta == 0 && tid == 0) record_status(BD_ERR_DEVICE_ARG);
+    return;
+  }
+  if (ps.W == 0) return;
+  const int64_t e0 = part_start(cta, ps.W, p.G), e1 = part_start(cta + 1, ps.W, p.G);
+  if (e1 <= e0) return;
+
+  const T *qg = static_cast<const T *>(p.q);
+  const T *kpg = static_cast<const T *>(p.k_prefix);
+  const T *vpg = static_cast<const T *>(p.v_prefix);
+  const T *kbg = static_cast<const T *>(p.k_blk);
+  const T *vbg = static_cast<const T *>(p.v_blk);
+  const int M = p.M, g = p.g;
+  const int64_t kstride = int64_t(p.H_kv) * D;  // elements between consecutive keys
+
+  constexpr int COLS4 = D / 4;      // lanes per output row
+  constexpr int PH = 32 / COLS4;    // rows handled at once per warp in P.V
+  constexpr int NI = 16 / PH;
+  const int c4 = lane % COLS4, ph = lane / COLS4;
+  const int nrw = (M - warp + 7) / 8;  // rows owned by this warp: warp + 8 i, i < nrw
+
+  int b = ps.b, cum_b = ps.cum_b;
+  int L = p.prefix_len[b];
+  int64_t off = p.prefix_offset[b];
+  int n = attn_units(L);
+  int kv = int((e0 - int64_t(p.H_kv) * cum_b) / n);
+  int64_t e = e0;
+
+  while (e < e1) {
+    const int64_t pbase = int64_t(p.H_kv) * cum_b + int64_t(kv) * n;
+    const int u0 = int(e - pbase);
+    const int u1 = int(e1 - pbase < int64_t(n) ? e1 - pbase : int64_t(n));
+    const bool first = (e == e0);
+    const bool complete = (u0 == 0 && u1 == n);
+
+    for (int idx = tid; idx < M * D; idx += kSimtThreads) {
+      const int m = idx / D, k = idx % D;
+      const int s = m / g, j = m % g;
+      Qs[m * D + k] = to_f32(qg[((int64_t(b) * p.S + s) * p.H_q + kv * g + j) * D + k]);
+    }
+    float mrow[16], lrow[16];
+    float acc[NI][4];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      mrow[i] = -INFINITY;
+      lrow[i] = 0.f;
+    }
+#pragma unroll
+    for (int i = 0; i < NI; ++i)
+#pragma unroll
+      for (int c = 0; c < 4; ++c) acc[i][c] = 0.f;
+    __syncthreads();
+
+    for (int u = u0; u < u1; ++u) {
+      const T *kbase, *vbase;
+      int cnt;
+      if (u < n - 1) {
+        const int64_t r0 = off + int64_t(u) * kUnitKeys;
+        cnt = min(kUnitKeys, L - u * kUnitKeys);
+        kbase = kpg + (r0 * p.H_kv + kv) * D;
+        vbase = vpg + (r0 * p.H_kv + kv) * D;
+      } else {
+        cnt = p.S;
+        kbase = kbg + (int64_t(b) * p.S * p.H_kv + kv) * D;
+        vbase = vbg + (int64_t(b) * p.S * p.H_kv + kv) * D;
+      }
+      for (int j0 = 0; j0 < cnt; j0 += kSimtKeys) {
+        const int nj = min(kSimtKeys, cnt - j0);
+        for (int idx = tid; idx < kSimtKeys * D; idx += kSimtThreads) {
+          const int j = idx / D, k = idx % D;
+          float kx = 0.f, vx = 0.f;
+          if (j < nj) {
+            kx = to_f32(kbase[int64_t(j0 + j) * kstride + k]);
+            vx = to_f32(vbase[int64_t(j0 + j) * kstride + k]);
+          }
+          Ks[j * (D + 4) + k] = kx;
+          Vs[j * D + k] = vx;
+        }
+        __syncthreads();
+
+        // scores of rows warp + 8 i against key `lane`
+        float sc[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) sc[i] = 0.f;
+        for (int k = 0; k < D; k += 4) {
+          const float4 kk = *reinterpret_cast<const float4 *>(&Ks[lane * (D + 4) + k]);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) {
+            if (i < nrw) {
+              const float4 qq = *reinterpret_cast<const float4 *>(&Qs[(warp + 8 * i) * D + k]);
+              sc[i] = fmaf(qq.x, kk.x, sc[i]);
+              sc[i] = fmaf(qq.y, kk.y, sc[i]);
+              sc[i] = fmaf(qq.z, kk.z, sc[i]);
+              sc[i] = fmaf(qq.w, kk.w, sc[i]);
+            }
+          }
+        }
+        // online softmax (base 2), one row at a time across the warp
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          if (i < nrw) {
+            const float x = (lane < nj) ? sc[i] * p.scale_log2 : -INFINITY;
+            const float mn = fmaxf(mrow[i], warp_max(x));
+            const float alpha = exp2f(mrow[i] - mn);
+            const float pv = exp2f(x - mn);
+            lrow[i] = lrow[i] * alpha + warp_sum(pv);
+            mrow[i] = mn;
+            Ps[(warp + 8 * i) * (kSimtKeys + 1) + lane] = pv;
+            if (lane == 0) s_alpha[warp + 8 * i] = alpha;
+          }
+        }
+        __syncwarp();
+        // P.V for rows warp + 8 (ph + PH i), columns 4 c4 .. 4 c4 + 3
+#pragma unroll
+        for (int i = 0; i < NI; ++i) {
+          const int ii = ph + PH * i;
+          if (ii < nrw) {
+            const float a = s_alpha[warp + 8 * ii];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) acc[i][c] *= a;
+          }
+        }
+        for (int j = 0; j < nj; ++j) {
+          const float4 v = *reinterpret_cast<const float4 *>(&Vs[j * D + 4 * c4]);
+#pragma unroll
+          for (int i = 0; i < NI; ++i) {
+            const int ii = ph + PH * i;
+            if (ii < nrw) {
+              const float pj = Ps[(warp + 8 * ii) * (kSimtKeys + 1) + j];
+              acc[i][0] = fmaf(pj, v.x, acc[i][0]);
+              acc[i][1] = fmaf(pj, v.y, acc[i][1]);
+              acc[i][2] = fmaf(pj, v.z, acc[i][2]);
+              acc[i][3] = fmaf(pj, v.w, acc[i][3]);
+            }
+          }
+        }
+        __syncthreads();
+      }
+    }
+
+    // segment result
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      if (i < nrw && lane == 0) {
+        s_l[warp + 8 * i] = lrow[i];
+        s_alpha[warp + 8 * i] = (mrow[i] + log2f(lrow[i])) * 0.69314718055994531f;
+      }
+    }
+    __syncwarp();
+#pragma unroll
+    for (int i = 0; i < NI; ++i) {
+      const int ii = ph + PH * i;
+      if (ii < nrw) {
+        const int m = warp + 8 * ii;
+        const float inv = 1.f / s_l[m];
+        const float4 r = make_float4(acc[i][0] * inv, acc[i][1] * inv, acc[i][2] * inv,
+                                     acc[i][3] * inv);
+        float *dst;
+        if (complete) {
+          const int s = m / g, j = m % g;
+          dst = p.o + ((int64_t(b) * p.S + s) * p.H_q + kv * g + j) * D;
+        } else {
+          dst = p.ws.slot + (attn_slot_index(cta, first) * M + m) * D;
+        }
+        *reinterpret_cast<float4 *>(dst + 4 * c4) = r;
+        if (c4 == 0) {
+          if (complete) {
+            const int s = m / g, j = m % g;
+            if (p.lse) p.lse[(int64_t(b) * p.H_q + kv * g + j) * p.S + s] = s_alpha[m];
+          } else {
+            p.ws.slot_lse[attn_slot_index(cta, first) * M + m] = s_alpha[m];
+          }
+        }
+      }
+    }
+
+    e = pbase + u1;
+    if (++kv == p.H_kv) {
+      kv = 0;
+      cum_b += n;
+      ++b;
+      if (b < p.B) {
+        L = p.prefix_len[b];
+        off = p.prefix_offset[b];
+        n = attn_units(L);
+      }
+    }
+    __syncthreads();
+  }
+}
+
+}  // namespace bd

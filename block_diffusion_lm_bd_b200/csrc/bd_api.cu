@@ -1,0 +1,279 @@
+// C ABI of libbd.so (declared in include/bd.h): host-side validation,
+// workspace layout, grid sizing and kernel launches. Everything that computes
+// runs in the kernels included below; this file only checks arguments and
+// launches.
+#include <atomic>
+#include <cmath>
+#include <cstdio>
+
+#include "attn_combine.cuh"
+#include "attn_simt.cuh"
+#include "unmask.cuh"
+
+namespace {
+
+std::atomic<uint64_t> g_launches{0};
+
+inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// SM count of the current device, or 0 when no device is usable.
+int sm_count() {
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  int n = 0;
+  if (cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+    cudaGetLastError();
+    return 0;
+  }
+  return n;
+}
+
+// Launch with programmatic stream serialisation: the kernel may be scheduled
+// while the previous kernel of the stream still runs; it waits for that
+// kernel's results with griddepcontrol.wait before reading them.
+template <typename Kern, typename Arg>
+cudaError_t launch_pdl(Kern kern, dim3 grid, dim3 block, size_t smem, cudaStream_t st,
+                       const Arg &arg) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, arg);
+}
+
+bd_status check_launch() {
+  g_launches.fetch_add(1, std::memory_order_relaxed);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) {
+    std::fprintf(stderr, "libbd: launch failed: %s\n", cudaGetErrorString(e));
+    return BD_ERR_CUDA;
+  }
+  return BD_OK;
+}
+
+bd_status attn_shape_ok(int B, int S, int H_q, int H_kv, int d) {
+  if (B < 0 || S < 1 || H_q < 1 || H_kv < 1) return BD_ERR_INVALID_ARG;
+  if (H_q % H_kv != 0) return BD_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return BD_ERR_UNSUPPORTED;
+  if (S > 64 || (H_q / H_kv) * S > bd::kMaxRows || B > bd::kMaxBatch) return BD_ERR_UNSUPPORTED;
+  return BD_OK;
+}
+
+int attn_grid(int sms) { return sms; }
+int unmask_grid(int sms) { return sms * bd::kUnmaskCtasPerSm; }
+
+}  // namespace
+
+extern "C" {
+
+int bd_version(void) { return 100; }
+
+const char *bd_status_string(bd_status s) {
+  switch (s) {
+    case BD_OK: return "BD_OK";
+    case BD_ERR_INVALID_ARG: return "BD_ERR_INVALID_ARG";
+    case BD_ERR_UNSUPPORTED: return "BD_ERR_UNSUPPORTED";
+    case BD_ERR_CUDA: return "BD_ERR_CUDA";
+    case BD_ERR_TIMEOUT: return "BD_ERR_TIMEOUT";
+    case BD_ERR_DEVICE_ARG: return "BD_ERR_DEVICE_ARG";
+  }
+  return "BD_ERR_UNKNOWN";
+}
+
+uint64_t bd_launch_count(void) { return g_launches.load(std::memory_order_relaxed); }
+
+size_t bd_attn_workspace_bytes(int B, int S, int H_q, int H_kv, int d) {
+  if (attn_shape_ok(B, S, H_q, H_kv, d) != BD_OK) return 0;
+  const int sms = sm_count();
+  if (sms <= 0) return 0;
+  const int M = (H_q / H_kv) * S;
+  return bd::attn_ws_layout(B, M, d, attn_grid(sms), nullptr, nullptr);
+}
+
+bd_status bd_attn_step(const void *q, const void *k_prefix, const void *v_prefix,
+                       int64_t prefix_rows, const void *k_blk, const void *v_blk,
+                       const int32_t *prefix_len, const int64_t *prefix_offset, int B, int S,
+                       int H_q, int H_kv, int d, float scale, bd_dtype dtype, float *o,
+                       float *lse, void *workspace, size_t workspace_bytes,
+                       bd_stream_t stream) {
+  bd_status st = attn_shape_ok(B, S, H_q, H_kv, d);
+  if (st != BD_OK) return st;
+  if (dtype != BD_DTYPE_F32 && dtype != BD_DTYPE_BF16) return BD_ERR_INVALID_ARG;
+  if (prefix_rows < 0 || prefix_rows > (int64_t(1) << 40)) return BD_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return BD_ERR_INVALID_ARG;
+  if (B == 0) return BD_OK;
+  if (!q || !k_blk || !v_blk || !o || !prefix_len || !prefix_offset || !workspace)
+    return BD_ERR_INVALID_ARG;
+  if (prefix_rows > 0 && (!k_prefix || !v_prefix)) return BD_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_blk) || !aligned16(v_blk) || !aligned16(o) ||
+      !aligned16(workspace) || (k_prefix && !aligned16(k_prefix)) ||
+      (v_prefix && !aligned16(v_prefix)) || (lse && !aligned16(lse)) ||
+      (reinterpret_cast<uintptr_t>(prefix_len) & 3u) ||
+      (reinterpret_cast<uintptr_t>(prefix_offset) & 7u))
+    return BD_ERR_INVALID_ARG;
+  const int sms = sm_count();
+  if (sms <= 0) return BD_ERR_CUDA;
+  const int G = attn_grid(sms);
+  const int g = H_q / H_kv, M = g * S;
+  if (workspace_bytes < bd::attn_ws_layout(B, M, d, G, nullptr, nullptr))
+    return BD_ERR_INVALID_ARG;
+
+  bd::AttnParams p = {};
+  p.q = q;
+  p.k_prefix = k_prefix;
+  p.v_prefix = v_prefix;
+  p.k_blk = k_blk;
+  p.v_blk = v_blk;
+  p.prefix_len = prefix_len;
+  p.prefix_offset = prefix_offset;
+  p.prefix_rows = prefix_rows;
+  p.B = B;
+  p.S = S;
+  p.H_q = H_q;
+  p.H_kv = H_kv;
+  p.d = d;
+  p.g = g;
+  p.M = M;
+  const float sc = scale > 0.f ? scale : 1.0f / std::sqrt(float(d));
+  p.scale_log2 = sc * 1.4426950408889634f;
+  p.o = o;
+  p.lse = lse;
+  bd::attn_ws_layout(B, M, d, G, &p.ws, static_cast<char *>(workspace));
+  p.G = G;
+  p.max_polls = bd::kDefaultMaxPolls;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+
+  {
+    void (*kern)(bd::AttnParams) = nullptr;
+    size_t smem = 0;
+    if (dtype == BD_DTYPE_F32) {
+      kern = d == 64 ? bd::attn_simt_kernel<float, 64> : bd::attn_simt_kernel<float, 128>;
+    } else {
+      kern = d == 64 ? bd::attn_simt_kernel<__nv_bfloat16, 64>
+                     : bd::attn_simt_kernel<__nv_bfloat16, 128>;
+    }
+    smem = d == 64 ? bd::simt_smem_bytes<64>() : bd::simt_smem_bytes<128>();
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
+        cudaSuccess) {
+      cudaGetLastError();
+      return BD_ERR_CUDA;
+    }
+    kern<<<G, bd::kSimtThreads, smem, cs>>>(p);
+    st = check_launch();
+    if (st != BD_OK) return st;
+  }
+  launch_pdl(bd::attn_combine_kernel, dim3(B * H_kv), dim3(bd::kCombineThreads), 0, cs, p);
+  return check_launch();
+}
+
+size_t bd_unmask_workspace_bytes(int rows, int V) {
+  if (rows < 0 || rows > bd::kUnmaskMaxRows || V < 1) return 0;
+  const int sms = sm_count();
+  if (sms <= 0) return 0;
+  return bd::unmask_ws_layout(rows, unmask_grid(sms), nullptr, nullptr);
+}
+
+bd_status bd_unmask(const float *logits, const uint8_t *mask, float gamma, int32_t *tokens_out,
+                    float *conf_out, uint8_t *commit_out, uint8_t *mask_out, int rows, int V,
+                    int block_S, int commit_at_least_one, void *workspace,
+                    size_t workspace_bytes, bd_stream_t stream) {
+  if (rows < 0 || rows > bd::kUnmaskMaxRows || V < 1) return BD_ERR_INVALID_ARG;
+  if (block_S < 0 || block_S > bd::kUnmaskFinalizeRows) return BD_ERR_INVALID_ARG;
+  if (commit_at_least_one && block_S < 1) return BD_ERR_INVALID_ARG;
+  if (std::isnan(gamma)) return BD_ERR_INVALID_ARG;
+  if (rows == 0) return BD_OK;
+  if (!logits || !mask || !tokens_out || !conf_out || !commit_out || !workspace)
+    return BD_ERR_INVALID_ARG;
+  if (!aligned16(logits) || !aligned16(workspace) ||
+      (reinterpret_cast<uintptr_t>(tokens_out) & 3u) ||
+      (reinterpret_cast<uintptr_t>(conf_out) & 3u))
+    return BD_ERR_INVALID_ARG;
+  const int sms = sm_count();
+  if (sms <= 0) return BD_ERR_CUDA;
+  const int G = unmask_grid(sms);
+  if (rows / G + 3 > bd::kUnmaskRowList) return BD_ERR_UNSUPPORTED;
+  if (workspace_bytes < bd::unmask_ws_layout(rows, G, nullptr, nullptr))
+    return BD_ERR_INVALID_ARG;
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+
+  bd::UnmaskParams rp = {};
+  rp.logits = logits;
+  rp.mask = mask;
+  rp.rows = rows;
+  rp.V = V;
+  rp.G = G;
+  bd::unmask_ws_layout(rows, G, &rp.ws, static_cast<char *>(workspace));
+  bd::unmask_reduce_kernel<<<G, bd::kUnmaskThreads, 0, cs>>>(rp);
+  bd_status st = check_launch();
+  if (st != BD_OK) return st;
+
+  bd::UnmaskFinalizeParams fp = {};
+  fp.mask = mask;
+  fp.gamma = gamma;
+  fp.tokens_out = tokens_out;
+  fp.conf_out = conf_out;
+  fp.commit_out = commit_out;
+  fp.mask_out = mask_out;
+  fp.rows = rows;
+  fp.V = V;
+  fp.G = G;
+  fp.block_S = block_S > 0 ? block_S : 1;
+  fp.fallback = commit_at_least_one ? 1 : 0;
+  fp.rows_per_cta = commit_at_least_one
+                        ? (bd::kUnmaskFinalizeRows / block_S) * block_S
+                        : bd::kUnmaskFinalizeRows;
+  fp.ws = rp.ws;
+  const int grid = (rows + fp.rows_per_cta - 1) / fp.rows_per_cta;
+  launch_pdl(bd::unmask_finalize_kernel, dim3(grid), dim3(bd::kUnmaskFinalizeRows), 0, cs, fp);
+  return check_launch();
+}
+
+bd_status bd_get_device_status(bd_stream_t stream) {
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(cs) != cudaSuccess) {
+    cudaGetLastError();
+    return BD_ERR_CUDA;
+  }
+  int s = 0;
+  if (cudaMemcpyFromSymbol(&s, bd::g_status, sizeof(int)) != cudaSuccess) {
+    cudaGetLastError();
+    return BD_ERR_CUDA;
+  }
+  const int zero = 0;
+  if (cudaMemcpyToSymbol(bd::g_status, &zero, sizeof(int)) != cudaSuccess) {
+    cudaGetLastError();
+    return BD_ERR_CUDA;
+  }
+  return static_cast<bd_status>(s);
+}
+
+}  // extern "C"
+
+namespace bd {
+// The only job of this kernel: wait, bounded, on a barrier nobody arrives on.
+__global__ void debug_wait_timeout_kernel(uint32_t max_polls) {
+  __shared__ __align__(8) uint64_t bar;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    fence_barrier_init();
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, max_polls);
+}
+}  // namespace bd
+
+extern "C" bd_status bd_debug_wait_timeout(int max_polls, bd_stream_t stream) {
+  if (max_polls < 0) return BD_ERR_INVALID_ARG;
+  bd::debug_wait_timeout_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
+      uint32_t(max_polls));
+  return check_launch();
+}

@@ -1,0 +1,142 @@
+// Shared device-side helpers of libbd: the device status word, bounded
+// barrier waits, the balanced work partition, and thin PTX wrappers for
+// mbarrier / TMA / tcgen05 on sm_100a.
+#pragma once
+
+#include <cuda.h>
+#include <cuda_bf16.h>
+#include <cuda_runtime.h>
+#include <stdint.h>
+
+#include "../../include/bd.h"
+
+namespace bd {
+
+// ---------------------------------------------------------------------------
+// Device status word: kernels record the first error they see; the host reads
+// and clears it with bd_get_device_status. One per device (a __device__
+// variable lives once per device per loaded module).
+// ---------------------------------------------------------------------------
+__device__ int g_status;
+
+__device__ __forceinline__ void record_status(int s) { atomicCAS(&g_status, 0, s); }
+
+// Default poll limit of every bounded wait (a poll costs >= ~32 ns with the
+// back-off below, so this is of the order of a second or more).
+constexpr uint32_t kDefaultMaxPolls = 1u << 25;
+
+// ---------------------------------------------------------------------------
+// Balanced partition of W work units over G workers: worker c owns
+// [start(c), start(c+1)) with start(c) = floor(c * W / G). Workers differ by at
+// most one unit; a range may cross item boundaries, which the kernels handle
+// by writing partial results.
+// ---------------------------------------------------------------------------
+__host__ __device__ __forceinline__ int64_t part_start(int64_t c, int64_t W, int64_t G) {
+  return (c * W) / G;
+}
+
+// Largest worker c with start(c) <= e (the worker that processes unit e).
+__host__ __device__ __forceinline__ int64_t part_owner(int64_t e, int64_t W, int64_t G) {
+  int64_t c = (e * G) / W;
+  if (c > G - 1) c = G - 1;
+  while (c + 1 < G && part_start(c + 1, W, G) <= e) ++c;
+  while (c > 0 && part_start(c, W, G) > e) --c;
+  return c;
+}
+
+// ---------------------------------------------------------------------------
+// mbarrier (shared-memory transaction barrier) helpers.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ uint32_t smem_u32(const void *p) {
+  return static_cast<uint32_t>(__cvta_generic_to_shared(p));
+}
+
+__device__ __forceinline__ void mbar_init(uint64_t *bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count));
+}
+
+__device__ __forceinline__ void fence_barrier_init() {
+  asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive(uint64_t *bar) {
+  asm volatile(
+      "{\n\t.reg .b64 st;\n\t"
+      "mbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(smem_u32(bar))
+      : "memory");
+}
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t *bar, uint32_t bytes) {
+  asm volatile(
+      "{\n\t.reg .b64 st;\n\t"
+      "mbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}" ::"r"(smem_u32(bar)),
+      "r"(bytes)
+      : "memory");
+}
+
+__device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t phase) {
+  uint32_t ok;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(phase)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait for the barrier phase with parity `phase` to complete. Returns
+// false (and records BD_ERR_TIMEOUT) after max_polls unsuccessful polls.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t phase, uint32_t max_polls) {
+  if (mbar_try_wait(bar, phase)) return true;
+  for (uint32_t i = 0; i < max_polls; ++i) {
+    if (mbar_try_wait(bar, phase)) return true;
+    if (i > 64) __nanosleep(32);
+  }
+  record_status(BD_ERR_TIMEOUT);
+  return false;
+}
+
+// ---------------------------------------------------------------------------
+// Misc.
+// ---------------------------------------------------------------------------
+__device__ __forceinline__ float warp_max(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v = fmaxf(v, __shfl_xor_sync(0xffffffffu, v, o));
+  return v;
+}
+
+__device__ __forceinline__ float warp_sum(float v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+__device__ __forceinline__ double warp_sum_d(double v) {
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) v += __shfl_xor_sync(0xffffffffu, v, o);
+  return v;
+}
+
+template <typename T>
+__device__ __forceinline__ float to_f32(T x);
+template <>
+__device__ __forceinline__ float to_f32<float>(float x) {
+  return x;
+}
+template <>
+__device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 x) {
+  return __bfloat162float(x);
+}
+
+// Programmatic dependent launch: let the next kernel in the stream start its
+// prologue early / wait for the previous kernel's results.
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+__device__ __forceinline__ void pdl_wait_previous() {
+  asm volatile("griddepcontrol.wait;" ::: "memory");
+}
+
+}  // namespace bd

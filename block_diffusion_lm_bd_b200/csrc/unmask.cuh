@@ -1,0 +1,311 @@
+// Confidence unmasking ("Technical summary: Nemotron-TwoTower", Training and
+// conditioning > Sampling, Algorithm 2): for every still-masked position, a
+// full-vocabulary softmax, its argmax token and that token's probability; the
+// position commits when the probability is higher than gamma.
+//
+// Two kernels:
+//  * unmask_reduce_kernel - a persistent grid (a multiple of the SM count)
+//    splits the logits of the masked rows, viewed as one stream of
+//    n_masked * V elements, into equal contiguous ranges. Each CTA streams its
+//    range once (16-byte loads, evict-first) and keeps per thread an online
+//    (max, argmax, sum of exp) with fp32 exponentials and an fp64 sum that is
+//    rescaled exactly whenever the running max grows. Rows wholly inside the
+//    CTA's range produce a final per-row record, rows cut by a range boundary
+//    a partial record in one of the CTA's two boundary slots.
+//  * unmask_finalize_kernel - per row: merge the records, confidence =
+//    1 / sum, commit = conf > gamma (decided in fp64), optional per-block
+//    fallback, write the outputs.
+#pragma once
+
+#include "bd_common.cuh"
+
+namespace bd {
+
+struct __align__(16) UnmaskPart {
+  double sum;  // sum over the segment of exp(l - m)
+  float m;     // max logit of the segment
+  int idx;     // lowest index attaining m
+};
+
+constexpr int kUnmaskThreads = 512;
+constexpr int kUnmaskCtasPerSm = 2;
+constexpr int kUnmaskMaxRows = 65536;
+constexpr int kUnmaskRowList = 1024;  // max rows one CTA's range can touch
+constexpr int kUnmaskFinalizeRows = 256;
+
+struct UnmaskWs {
+  int *n_masked;         // [1]
+  int *rank;             // [rows]  rank among masked rows, -1 if unmasked
+  UnmaskPart *row_part;  // [rows]  rows finished inside one CTA
+  UnmaskPart *slot;      // [G][2]  first / last cut segment of each CTA
+};
+
+__host__ __device__ inline size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+__host__ __device__ inline size_t unmask_ws_layout(int rows, int G, UnmaskWs *ws, char *base) {
+  size_t off = 0;
+  if (ws) ws->n_masked = reinterpret_cast<int *>(base + off);
+  off = align256(off + sizeof(int));
+  if (ws) ws->rank = reinterpret_cast<int *>(base + off);
+  off = align256(off + sizeof(int) * size_t(rows));
+  if (ws) ws->row_part = reinterpret_cast<UnmaskPart *>(base + off);
+  off = align256(off + sizeof(UnmaskPart) * size_t(rows));
+  if (ws) ws->slot = reinterpret_cast<UnmaskPart *>(base + off);
+  off = align256(off + sizeof(UnmaskPart) * size_t(G) * 2);
+  return off;
+}
+
+struct UnmaskParams {
+  const float *logits;
+  const uint8_t *mask;
+  int rows;
+  int V;
+  int G;
+  UnmaskWs ws;
+};
+
+// Fold one value at index i into a thread's running (m, idx, s).
+__device__ __forceinline__ void um_fold1(float x, int i, float &m, int &idx, double &s) {
+  if (x > m) {
+    s = (m == -INFINITY) ? 0.0 : s * exp(double(m) - double(x));
+    m = x;
+    idx = i;
+  }
+  s += double(expf(x - m));
+}
+
+// Fold four consecutive values starting at index i.
+__device__ __forceinline__ void um_fold4(float4 x, int i, float &m, int &idx, double &s) {
+  float gm = fmaxf(fmaxf(x.x, x.y), fmaxf(x.z, x.w));
+  if (gm > m) {
+    s = (m == -INFINITY) ? 0.0 : s * exp(double(m) - double(gm));
+    m = gm;
+    idx = i + (x.x == gm ? 0 : (x.y == gm ? 1 : (x.z == gm ? 2 : 3)));
+  }
+  float e = (expf(x.x - m) + expf(x.y - m)) + (expf(x.z - m) + expf(x.w - m));
+  s += double(e);
+}
+
+// Block-wide merge of the per-thread (m, idx, s); result valid in thread 0.
+__device__ __forceinline__ UnmaskPart um_block_reduce(float m, int idx, double s, float *sm_m,
+                                                      int *sm_i, double *sm_s) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nwarps = blockDim.x >> 5;
+  float wm = warp_max(m);
+  if (lane == 0) sm_m[warp] = wm;
+  __syncthreads();
+  float M = -INFINITY;
+  for (int w = 0; w < nwarps; ++w) M = fmaxf(M, sm_m[w]);
+  double sc = (m == -INFINITY) ? 0.0 : s * exp(double(m) - double(M));
+  int ic = (m == M) ? idx : INT_MAX;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) {
+    sc += __shfl_xor_sync(0xffffffffu, sc, o);
+    ic = min(ic, __shfl_xor_sync(0xffffffffu, ic, o));
+  }
+  if (lane == 0) {
+    sm_s[warp] = sc;
+    sm_i[warp] = ic;
+  }
+  __syncthreads();
+  UnmaskPart r;
+  r.m = M;
+  r.sum = 0.0;
+  r.idx = INT_MAX;
+  if (threadIdx.x == 0) {
+    for (int w = 0; w < nwarps; ++w) {
+      r.sum += sm_s[w];
+      r.idx = min(r.idx, sm_i[w]);
+    }
+  }
+  __syncthreads();
+  return r;
+}
+
+__global__ void __launch_bounds__(kUnmaskThreads, kUnmaskCtasPerSm)
+    unmask_reduce_kernel(UnmaskParams p) {
+  __shared__ int s_cnt[kUnmaskThreads];
+  __shared__ int s_rows[kUnmaskRowList];
+  __shared__ float sm_m[32];
+  __shared__ int sm_i[32];
+  __shared__ double sm_s[32];
+  __shared__ int s_total;
+
+  const int tid = threadIdx.x;
+  const int c = blockIdx.x;
+  // Let the finalize kernel get launched while this grid runs.
+  pdl_launch_dependents();
+
+  // 1. Ranks of the masked rows: each thread counts a contiguous chunk.
+  const int chunk = (p.rows + kUnmaskThreads - 1) / kUnmaskThreads;
+  const int r_lo = min(p.rows, tid * chunk), r_hi = min(p.rows, r_lo + chunk);
+  int cnt = 0;
+  for (int r = r_lo; r < r_hi; ++r) cnt += (p.mask[r] != 0);
+  s_cnt[tid] = cnt;
+  __syncthreads();
+  // Inclusive scan (Hillis-Steele) over the per-thread counts.
+  for (int o = 1; o < kUnmaskThreads; o <<= 1) {
+    int v = (tid >= o) ? s_cnt[tid - o] : 0;
+    __syncthreads();
+    s_cnt[tid] += v;
+    __syncthreads();
+  }
+  const int excl = s_cnt[tid] - cnt;
+  if (tid == kUnmaskThreads - 1) s_total = s_cnt[tid];
+  __syncthreads();
+  const int n_masked = s_total;
+  const int64_t V = p.V;
+  const int64_t W = int64_t(n_masked) * V;
+  const int64_t G = p.G;
+  const int64_t e0 = W ? part_start(c, W, G) : 0, e1 = W ? part_start(c + 1, W, G) : 0;
+  const int64_t rho0 = e0 / V;
+  const int64_t rho1 = (e1 > e0) ? (e1 - 1) / V : rho0 - 1;
+
+  // Row list of this CTA's range; CTA 0 also publishes all ranks.
+  {
+    int rk = excl;
+    for (int r = r_lo; r < r_hi; ++r) {
+      const bool mk = p.mask[r] != 0;
+      if (c == 0) p.ws.rank[r] = mk ? rk : -1;
+      if (mk) {
+        if (rk >= rho0 && rk <= rho1) s_rows[rk - rho0] = r;
+        ++rk;
+      }
+    }
+    if (c == 0 && tid == 0) *p.ws.n_masked = n_masked;
+  }
+  __syncthreads();
+  if (e1 <= e0) return;
+
+  // 2. Stream every segment of the range.
+  for (int64_t rho = rho0; rho <= rho1; ++rho) {
+    const int row = s_rows[rho - rho0];
+    const int64_t rs = rho * V;
+    const int v0 = int(max(e0, rs) - rs);
+    const int v1 = int(min(e1, rs + V) - rs);
+    const float *x = p.logits + int64_t(row) * V;
+    float m = -INFINITY;
+    int idx = INT_MAX;
+    double s = 0.0;
+    // head: scalar up to 16-byte alignment
+    const int mis = int((reinterpret_cast<uintptr_t>(x + v0) >> 2) & 3);
+    const int head = min(v1 - v0, (4 - mis) & 3);
+    if (tid < head) um_fold1(__ldcs(x + v0 + tid), v0 + tid, m, idx, s);
+    const int b0 = v0 + head;
+    const int ng = (v1 - b0) >> 2;
+    const float4 *x4 = reinterpret_cast<const float4 *>(x + b0);
+    int g = tid;
+    for (; g + 3 * kUnmaskThreads < ng; g += 4 * kUnmaskThreads) {
+      float4 a0 = __ldcs(x4 + g);
+      float4 a1 = __ldcs(x4 + g + kUnmaskThreads);
+      float4 a2 = __ldcs(x4 + g + 2 * kUnmaskThreads);
+      float4 a3 = __ldcs(x4 + g + 3 * kUnmaskThreads);
+      um_fold4(a0, b0 + 4 * g, m, idx, s);
+      um_fold4(a1, b0 + 4 * (g + kUnmaskThreads), m, idx, s);
+      um_fold4(a2, b0 + 4 * (g + 2 * kUnmaskThreads), m, idx, s);
+      um_fold4(a3, b0 + 4 * (g + 3 * kUnmaskThreads), m, idx, s);
+    }
+    for (; g < ng; g += kUnmaskThreads) um_fold4(__ldcs(x4 + g), b0 + 4 * g, m, idx, s);
+    const int t0 = b0 + 4 * ng;
+    if (t0 + tid < v1) um_fold1(__ldcs(x + t0 + tid), t0 + tid, m, idx, s);
+
+    UnmaskPart r = um_block_reduce(m, idx, s, sm_m, sm_i, sm_s);
+    if (tid == 0) {
+      if (v0 == 0 && v1 == V)
+        p.ws.row_part[row] = r;
+      else
+        p.ws.slot[2 * int64_t(c) + (rho == rho0 ? 0 : 1)] = r;
+    }
+  }
+}
+
+struct UnmaskFinalizeParams {
+  const uint8_t *mask;
+  float gamma;
+  int32_t *tokens_out;
+  float *conf_out;
+  uint8_t *commit_out;
+  uint8_t *mask_out;
+  int rows;
+  int V;
+  int G;
+  int block_S;
+  int fallback;
+  int rows_per_cta;
+  UnmaskWs ws;
+};
+
+__device__ __forceinline__ void um_merge(UnmaskPart &a, const UnmaskPart &b) {
+  if (b.m > a.m) {
+    a.sum = a.sum * exp(double(a.m) - double(b.m)) + b.sum;
+    a.m = b.m;
+    a.idx = b.idx;
+  } else if (b.m < a.m) {
+    a.sum += b.sum * exp(double(b.m) - double(a.m));
+  } else {
+    a.sum += b.sum;
+    a.idx = min(a.idx, b.idx);
+  }
+}
+
+__global__ void __launch_bounds__(kUnmaskFinalizeRows)
+    unmask_finalize_kernel(UnmaskFinalizeParams p) {
+  __shared__ double s_conf[kUnmaskFinalizeRows];
+  __shared__ uint8_t s_commit[kUnmaskFinalizeRows];
+  __shared__ uint8_t s_mask[kUnmaskFinalizeRows];
+  pdl_wait_previous();
+  const int r = blockIdx.x * p.rows_per_cta + threadIdx.x;
+  const bool in = threadIdx.x < p.rows_per_cta && r < p.rows;
+  uint8_t mk = in ? (p.mask[r] != 0) : 0;
+  uint8_t commit = 0;
+  double conf = -1.0;
+  if (mk) {
+    const int64_t V = p.V, G = p.G;
+    const int64_t W = int64_t(*p.ws.n_masked) * V;
+    const int64_t e0 = int64_t(p.ws.rank[r]) * V, e1 = e0 + V;
+    const int64_t c0 = part_owner(e0, W, G), c1 = part_owner(e1 - 1, W, G);
+    UnmaskPart a;
+    if (c0 == c1) {
+      a = p.ws.row_part[r];
+    } else {
+      a = p.ws.slot[2 * c0 + (part_start(c0, W, G) == e0 ? 0 : 1)];
+      for (int64_t c = c0 + 1; c <= c1; ++c)
+        if (part_start(c, W, G) < part_start(c + 1, W, G)) um_merge(a, p.ws.slot[2 * c]);
+    }
+    conf = 1.0 / a.sum;
+    commit = conf > double(p.gamma);
+    p.tokens_out[r] = a.idx;
+    p.conf_out[r] = float(conf);
+  }
+  if (p.fallback) {
+    s_conf[threadIdx.x] = conf;
+    s_commit[threadIdx.x] = commit;
+    s_mask[threadIdx.x] = mk;
+    __syncthreads();
+    // the first row of each block decides for its block
+    const int lr = threadIdx.x;
+    if (in && lr % p.block_S == 0) {
+      const int n = min(p.block_S, p.rows_per_cta - lr);
+      bool any_masked = false, any_commit = false;
+      int best = -1;
+      double bc = -1.0;
+      for (int k = 0; k < n && r + k < p.rows; ++k) {
+        any_masked |= s_mask[lr + k] != 0;
+        any_commit |= s_commit[lr + k] != 0;
+        if (s_mask[lr + k] && s_conf[lr + k] > bc) {
+          bc = s_conf[lr + k];
+          best = lr + k;
+        }
+      }
+      if (any_masked && !any_commit && best >= 0) s_commit[best] = 1;
+    }
+    __syncthreads();
+    commit = s_commit[threadIdx.x];
+  }
+  if (in) {
+    p.commit_out[r] = commit;
+    if (p.mask_out) p.mask_out[r] = (mk && !commit) ? 1 : 0;
+  }
+}
+
+}  // namespace bd

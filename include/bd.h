@@ -1,0 +1,191 @@
+/*
+ * bd.h - C ABI of libbd.so: one denoising step of a block-diffusion LM on
+ * NVIDIA B200 (sm_100a).
+ *
+ * The step has two parts, both defined on the source pages:
+ *
+ *  1. bd_attn_step - the S queries of the active block attend to a cached
+ *     clean-prefix KV and, bidirectionally, to the block's own KV, merged in
+ *     one softmax ("Technical summary: Nemotron-TwoTower", Methodology >
+ *     Architecture, item 2, and Methodology > Generation process, third
+ *     bullet). The prefix cache is read-only: it depends on the clean prefix
+ *     only ("Training Hybrid Block Diffusion Language Models with Partial
+ *     Bidirectionality", Methodology, cache-aligned objective).
+ *
+ *  2. bd_unmask - confidence unmasking ("Technical summary:
+ *     Nemotron-TwoTower", Training and conditioning > Sampling, Algorithm 2):
+ *     every masked position gets a full-vocabulary softmax; its argmax token
+ *     and that token's probability (the confidence); positions whose
+ *     confidence is higher than gamma commit.
+ *
+ * Conventions shared by every call:
+ *  - Every pointer is caller-owned DEVICE memory (the library allocates
+ *    nothing and frees nothing). Inputs are never written.
+ *  - Every call is asynchronous on `stream` (NULL = the legacy default
+ *    stream); nothing synchronises except bd_get_device_status.
+ *  - The return value reports host-side validation (before any launch) and
+ *    launch errors. Errors found on the device (bad offsets inside device
+ *    arrays, a bounded wait that ran out) are recorded in a per-process
+ *    device status word read by bd_get_device_status.
+ *  - Pointers must be 16-byte aligned. Tensors are dense, row-major (last
+ *    index fastest), with exactly the strides implied by their shapes.
+ *  - Inputs must be finite (no NaN / Inf).
+ *  - The calls are re-entrant per stream: two calls that share a workspace
+ *    must not run concurrently on different streams.
+ */
+#ifndef BD_H_
+#define BD_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* Same type as cudaStream_t. */
+typedef struct CUstream_st *bd_stream_t;
+
+typedef enum {
+  BD_OK = 0,
+  BD_ERR_INVALID_ARG = 1, /* a pointer, size or shape is invalid            */
+  BD_ERR_UNSUPPORTED = 2, /* valid, but outside what the kernels implement  */
+  BD_ERR_CUDA = 3,        /* a CUDA runtime / driver call or launch failed  */
+  BD_ERR_TIMEOUT = 4,     /* device: a bounded wait ran out (kernel exited) */
+  BD_ERR_DEVICE_ARG = 5   /* device: prefix_len / prefix_offset out of range */
+} bd_status;
+
+typedef enum { BD_DTYPE_F32 = 0, BD_DTYPE_BF16 = 1 } bd_dtype;
+
+/* Library version, e.g. 100 for 1.0.0. */
+int bd_version(void);
+
+/* Human-readable name of a status code (static string, never NULL). */
+const char *bd_status_string(bd_status s);
+
+/* ------------------------------------------------------------------------ */
+/* Attention of the active block over prefix ++ block keys                 */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Workspace bytes bd_attn_step needs on the CURRENT device for these sizes
+ * (it depends on the device's SM count). Returns 0 if the sizes are invalid
+ * or no CUDA device is usable. The workspace holds per-split partial results
+ * (normalised outputs and log-sum-exps) and needs no initialisation.
+ */
+size_t bd_attn_workspace_bytes(int B, int S, int H_q, int H_kv, int d);
+
+/*
+ * One attention step for B sequences (one layer).
+ *
+ * For every sequence b, query head h (KV head kv = h / (H_q/H_kv): grouped
+ * query heads map contiguously) and block position i:
+ *     keys   = k_prefix[prefix_offset[b] + 0 .. prefix_len[b]-1, kv, :]
+ *              ++ k_blk[b, 0 .. S-1, kv, :]
+ *     values = the same rows of v_prefix ++ v_blk
+ *     o[b,i,h,:]  = softmax(keys . q[b,i,h,:] * scale) . values
+ *     lse[b,h,i]  = natural log of sum(exp(keys . q[b,i,h,:] * scale))
+ * Every block query sees every prefix key of its sequence (the prefix lies
+ * wholly in the past) and every key of its own block (bidirectional, no
+ * mask). No position encoding is applied here.
+ *
+ * Arguments (all device pointers unless said otherwise):
+ *   q            [B, S, H_q, d]         dtype
+ *   k_prefix     [prefix_rows, H_kv, d] dtype, packed rows of all sequences
+ *   v_prefix     [prefix_rows, H_kv, d] dtype
+ *   prefix_rows  number of rows allocated in k_prefix / v_prefix (host int)
+ *   k_blk, v_blk [B, S, H_kv, d]        dtype
+ *   prefix_len   int32 [B], >= 0: valid prefix rows of sequence b
+ *   prefix_offset int64 [B] (or longer): first row of sequence b; rows
+ *                offset .. offset+len-1 must lie in [0, prefix_rows)
+ *   scale        score scale; <= 0 selects 1/sqrt(d)
+ *   dtype        BD_DTYPE_BF16 (tensor-core path) or BD_DTYPE_F32
+ *   o            float32 [B, S, H_q, d]  output
+ *   lse          float32 [B, H_q, S]     output, or NULL
+ *   workspace    >= bd_attn_workspace_bytes(B, S, H_q, H_kv, d) bytes
+ * Supported: d in {64, 128}; 1 <= S <= 64; H_q % H_kv == 0;
+ * (H_q/H_kv) * S <= 128; B <= 65535. Otherwise BD_ERR_UNSUPPORTED /
+ * BD_ERR_INVALID_ARG, and nothing is launched. Offsets or lengths out of
+ * range are found on the device: nothing is written and the device status
+ * becomes BD_ERR_DEVICE_ARG.
+ */
+bd_status bd_attn_step(const void *q, const void *k_prefix, const void *v_prefix,
+                       int64_t prefix_rows, const void *k_blk, const void *v_blk,
+                       const int32_t *prefix_len, const int64_t *prefix_offset, int B, int S,
+                       int H_q, int H_kv, int d, float scale, bd_dtype dtype, float *o,
+                       float *lse, void *workspace, size_t workspace_bytes,
+                       bd_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Confidence unmasking                                                     */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Workspace bytes bd_unmask needs on the CURRENT device (depends on its SM
+ * count). Returns 0 for invalid sizes or when no CUDA device is usable. No
+ * initialisation is needed.
+ */
+size_t bd_unmask_workspace_bytes(int rows, int V);
+
+/*
+ * Confidence unmasking of `rows` positions over a vocabulary of V tokens.
+ *
+ * For every row r with mask[r] != 0 (still masked):
+ *     tokens_out[r] = the argmax token of logits[r, :] (lowest id on ties)
+ *     conf_out[r]   = its softmax probability = 1 / sum_v exp(l_rv - max_v l_rv)
+ *                     (exponentials in float32, sums in float64, stored as float32)
+ *     commit_out[r] = conf > gamma (strict; decided in float64 against the
+ *                     float32 gamma)
+ * Optional fallback (commit_at_least_one != 0, block_S > 0): rows are grouped
+ * in blocks of block_S consecutive rows; a block that still has masked rows
+ * and commits none commits its masked row of highest confidence (lowest row
+ * on ties). This rule is a build assumption, not from the pages.
+ * For rows with mask[r] == 0: the logits are not read, tokens_out / conf_out
+ * are left untouched and commit_out[r] = 0.
+ * mask_out (optional, may be NULL or equal to mask): mask && !commit.
+ *
+ *   logits      float32 [rows, V]
+ *   mask        uint8   [rows]
+ *   tokens_out  int32   [rows]
+ *   conf_out    float32 [rows]
+ *   commit_out  uint8   [rows]
+ *   mask_out    uint8   [rows] or NULL
+ * Supported: 1 <= rows <= 65536, 1 <= V < 2^31, block_S in [0, 1024].
+ */
+bd_status bd_unmask(const float *logits, const uint8_t *mask, float gamma, int32_t *tokens_out,
+                    float *conf_out, uint8_t *commit_out, uint8_t *mask_out, int rows, int V,
+                    int block_S, int commit_at_least_one, void *workspace,
+                    size_t workspace_bytes, bd_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Status, diagnostics                                                      */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Synchronises `stream`, then returns and clears the device status word of
+ * the current device (BD_OK if no kernel recorded an error). A CUDA error
+ * seen while synchronising returns BD_ERR_CUDA.
+ */
+bd_status bd_get_device_status(bd_stream_t stream);
+
+/*
+ * Number of kernels this process has launched through the library so far
+ * (host-side counter, all devices). Lets a caller count the kernels of a
+ * timed region.
+ */
+uint64_t bd_launch_count(void);
+
+/*
+ * Test hook for the failure path: launches one tiny kernel whose only job is
+ * a bounded wait on a shared-memory barrier that nothing ever arrives on.
+ * The wait gives up after `max_polls` polls, records BD_ERR_TIMEOUT in the
+ * device status word and returns, leaving the context usable. Read the
+ * result with bd_get_device_status.
+ */
+bd_status bd_debug_wait_timeout(int max_polls, bd_stream_t stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* BD_H_ */

@@ -99,5 +99,7 @@ def top2_gap(logits):
     implementations that round differently; parity reports them separately.
     """
     x = _f64(logits)
+    if x.shape[1] < 2:  # one token: no runner-up, the argmax is unique
+        return np.full(x.shape[0], np.inf)
     part = np.partition(x, x.shape[1] - 2, axis=1)
     return part[:, -1] - part[:, -2]

@@ -1,0 +1,61 @@
+"""Shared helpers of the parity tests (comparison rules, not arithmetic of the step)."""
+
+import numpy as np
+import torch
+
+from oracle.unmask import top2_gap
+
+# Attention tolerance: max |o_gpu - o_ref| divided by the standard deviation of
+# o_ref over the compared elements ("relative to unit-variance outputs").
+ATTN_TOL = {torch.bfloat16: 2e-2, torch.float32: 1e-4}
+LSE_TOL = {torch.bfloat16: 2e-3, torch.float32: 1e-5}
+# Unmask: token ids and commits bit-exact, except rows whose top-2 logits differ
+# by < 1e-6 (token) or whose confidence lies within 1e-6 of gamma (commit).
+NEAR = 1e-6
+CONF_TOL = 1e-6
+
+
+def attn_err(o_gpu, o_ref):
+    o_gpu = np.asarray(o_gpu, dtype=np.float64)
+    o_ref = np.asarray(o_ref, dtype=np.float64)
+    sd = o_ref.std()
+    return float(np.abs(o_gpu - o_ref).max() / sd), float(np.abs(o_gpu - o_ref).max())
+
+
+def to_np(t):
+    return t.detach().to("cpu").to(torch.float64).numpy() if t.is_floating_point() else \
+        t.detach().to("cpu").numpy()
+
+
+def compare_unmask(res_gpu, ref, logits, mask, gamma, block_S=None, fallback=False):
+    """Check GPU unmask outputs against the oracle's. Returns exclusion counts."""
+    tok = res_gpu["tokens"].cpu().numpy().astype(np.int64)
+    conf = res_gpu["conf"].cpu().numpy().astype(np.float64)
+    commit = res_gpu["commit"].cpu().numpy().astype(bool)
+    m = np.asarray(mask.cpu().numpy() if hasattr(mask, "cpu") else mask).astype(bool)
+    gap = top2_gap(logits)
+    thr = float(np.float32(gamma))
+    near_tie = m & (gap < NEAR)
+    near_gamma = m & (np.abs(np.nan_to_num(ref["conf"], nan=-1.0) - thr) < NEAR)
+    ok_tok = m & ~near_tie
+    assert (tok[ok_tok] == ref["tokens"][ok_tok]).all(), \
+        f"token mismatch at rows {np.flatnonzero(ok_tok & (tok != ref['tokens']))[:10]}"
+    assert np.abs(conf[m] - ref["conf"][m]).max(initial=0.0) <= CONF_TOL
+    excluded_blocks = np.zeros(len(m), dtype=bool)
+    if fallback:
+        # a block whose fallback choice hinges on two confidences within 1e-6
+        for s in range(0, len(m), block_S):
+            sl = slice(s, min(s + block_S, len(m)))
+            c = np.where(m[sl], ref["conf"][sl], -np.inf)
+            if m[sl].sum() >= 2:
+                top = np.sort(c)[-2:]
+                if np.isfinite(top).all() and top[1] - top[0] < NEAR:
+                    excluded_blocks[sl] = True
+            if near_gamma[sl].any():
+                excluded_blocks[sl] = True
+    ok_c = ~near_gamma & ~excluded_blocks
+    bad = np.flatnonzero(ok_c & (commit != ref["commit"]))
+    assert bad.size == 0, f"commit mismatch at rows {bad[:10]}"
+    assert not commit[~m].any()
+    return {"near_tie": int(near_tie.sum()), "near_gamma": int(near_gamma.sum()),
+            "excluded_blocks_rows": int(excluded_blocks.sum())}

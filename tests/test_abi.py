@@ -1,0 +1,146 @@
+"""The C ABI without a GPU: the library loads, exports every function bd.h
+declares, and rejects invalid arguments on the host before any launch."""
+
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+import torch
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "bd.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    from block_diffusion_lm_bd_b200 import build
+
+    build.build()
+    from block_diffusion_lm_bd_b200 import api
+
+    return api._lib()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(bd_[a-z_0-9]+)\s*\(", src)))
+
+
+def test_header_declares_the_boundary():
+    names = declared_functions()
+    for required in ("bd_attn_step", "bd_attn_workspace_bytes", "bd_unmask",
+                     "bd_unmask_workspace_bytes", "bd_get_device_status", "bd_status_string"):
+        assert required in names
+
+
+def test_every_declared_symbol_is_exported(lib):
+    path = os.path.join(ROOT, "block_diffusion_lm_bd_b200", "libbd.so")
+    out = subprocess.run(["nm", "-D", "--defined-only", path], capture_output=True, text=True).stdout
+    exported = set(re.findall(r"\b[TW] (bd_[a-z_0-9]+)\b", out))
+    missing = [n for n in declared_functions() if n not in exported]
+    assert not missing, f"declared but not exported: {missing}"
+    for n in declared_functions():
+        getattr(lib, n)  # resolvable through ctypes too
+
+
+def test_status_strings(lib):
+    from block_diffusion_lm_bd_b200 import api
+
+    assert api.status_string(0) == "BD_OK"
+    assert api.status_string(4) == "BD_ERR_TIMEOUT"
+    assert api.status_string(5) == "BD_ERR_DEVICE_ARG"
+    assert api.status_string(99) == "BD_ERR_UNKNOWN"
+    assert lib.bd_version() >= 100
+
+
+def _attn(lib, **kw):
+    a = dict(q=16, kp=16, vp=16, rows=10, kb=16, vb=16, pl=16, po=16, B=2, S=16, Hq=8, Hkv=2, d=64,
+             scale=0.0, dtype=0, o=16, lse=0, ws=16, wsb=1 << 30, st=0)
+    a.update(kw)
+    vp = lambda x: ctypes.c_void_p(x) if x else None
+    return lib.bd_attn_step(vp(a["q"]), vp(a["kp"]), vp(a["vp"]), a["rows"], vp(a["kb"]), vp(a["vb"]),
+                            vp(a["pl"]), vp(a["po"]), a["B"], a["S"], a["Hq"], a["Hkv"], a["d"],
+                            a["scale"], a["dtype"], vp(a["o"]), vp(a["lse"]), vp(a["ws"]),
+                            a["wsb"], vp(a["st"]))
+
+
+INVALID, UNSUPPORTED, CUDA = 1, 2, 3
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(d=96), UNSUPPORTED),
+    (dict(S=65), UNSUPPORTED),
+    (dict(S=0), INVALID),
+    (dict(Hq=6, Hkv=4), INVALID),
+    (dict(Hq=32, Hkv=2, S=16), UNSUPPORTED),      # g*S = 256 rows > 128
+    (dict(B=5000), UNSUPPORTED),
+    (dict(B=-1), INVALID),
+    (dict(q=0), INVALID),
+    (dict(o=0), INVALID),
+    (dict(ws=0), INVALID),
+    (dict(pl=0), INVALID),
+    (dict(kp=0), INVALID),                       # prefix rows > 0 need k_prefix
+    (dict(q=24), INVALID),                       # misaligned
+    (dict(po=20), INVALID),                      # int64 array misaligned
+    (dict(dtype=7), INVALID),
+    (dict(rows=-3), INVALID),
+    (dict(scale=float("nan")), INVALID),
+])
+def test_attn_host_validation(lib, kw, code):
+    assert _attn(lib, **kw) == code
+
+
+def test_attn_empty_batch_is_a_no_op(lib):
+    assert _attn(lib, B=0) == 0
+
+
+def _unmask(lib, **kw):
+    a = dict(lg=16, mk=16, gamma=0.9, tok=16, conf=16, com=16, mo=0, rows=4, V=8, bs=0, fb=0,
+             ws=16, wsb=1 << 30, st=0)
+    a.update(kw)
+    vp = lambda x: ctypes.c_void_p(x) if x else None
+    return lib.bd_unmask(vp(a["lg"]), vp(a["mk"]), a["gamma"], vp(a["tok"]), vp(a["conf"]),
+                         vp(a["com"]), vp(a["mo"]), a["rows"], a["V"], a["bs"], a["fb"],
+                         vp(a["ws"]), a["wsb"], vp(a["st"]))
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(rows=-1), INVALID),
+    (dict(rows=70000), INVALID),
+    (dict(V=0), INVALID),
+    (dict(bs=-1), INVALID),
+    (dict(bs=300), INVALID),
+    (dict(fb=1, bs=0), INVALID),
+    (dict(lg=0), INVALID),
+    (dict(mk=0), INVALID),
+    (dict(tok=0), INVALID),
+    (dict(ws=0), INVALID),
+    (dict(lg=20), INVALID),
+    (dict(gamma=float("nan")), INVALID),
+])
+def test_unmask_host_validation(lib, kw, code):
+    assert _unmask(lib, **kw) == code
+
+
+def test_unmask_zero_rows_is_a_no_op(lib):
+    assert _unmask(lib, rows=0) == 0
+
+
+@pytest.mark.skipif(torch.cuda.is_available(), reason="checks the no-GPU behaviour")
+def test_without_gpu_sizes_are_zero_and_calls_fail_cleanly(lib):
+    assert lib.bd_attn_workspace_bytes(1, 16, 8, 2, 64) == 0
+    assert lib.bd_unmask_workspace_bytes(16, 1024) == 0
+    assert _attn(lib) == CUDA  # passes host validation, then finds no device
+
+
+def test_product_package_never_imports_the_oracle():
+    pkg = os.path.join(ROOT, "block_diffusion_lm_bd_b200")
+    for dirpath, _, files in os.walk(pkg):
+        for f in files:
+            if f.endswith((".py", ".cu", ".cuh", ".h")):
+                src = open(os.path.join(dirpath, f)).read()
+                assert not re.search(r"^\s*(from|import)\s+oracle\b", src, re.M), f
+                assert "oracle/" not in src, f

@@ -1,0 +1,149 @@
+"""GPU parity of bd_attn_step (through the C ABI) against the float64 oracle.
+
+Bar: max |o_gpu - o_ref| / std(o_ref) <= 2e-2 for bf16 inputs and 1e-4 for
+fp32 inputs; lse within 2e-3 (bf16) / 1e-5 (fp32) absolute. Small cases are
+compared element by element over several work units and ragged tails; the
+full-size workloads on sampled output rows the oracle computes one by one.
+"""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from block_diffusion_lm_bd_b200 import api, workloads
+from oracle.attention import block_attention, block_attention_rows
+from _util import ATTN_TOL, LSE_TOL, attn_err, to_np
+
+pytestmark = pytest.mark.gpu
+DEV = torch.device("cuda", 0)
+
+
+def _gpu(inp, scale=None):
+    o, lse = api.attn_step(inp["q"], inp["k_prefix"], inp["v_prefix"], inp["k_blk"], inp["v_blk"],
+                           inp["prefix_len"], inp["prefix_offset"], scale=scale)
+    torch.cuda.synchronize()
+    st = api.get_device_status()
+    assert st == 0, api.status_string(st)
+    return o, lse
+
+
+def _full_check(inp, dtype, scale=None):
+    o, lse = _gpu(inp, scale)
+    ro, rl = block_attention(inp["q"], inp["k_prefix"], inp["v_prefix"], inp["k_blk"],
+                             inp["v_blk"], inp["prefix_len_host"], inp["prefix_offset_host"],
+                             scale=scale)
+    err, raw = attn_err(to_np(o), ro)
+    lerr = float(np.abs(to_np(lse) - rl).max())
+    assert err <= ATTN_TOL[dtype], (err, raw)
+    assert lerr <= LSE_TOL[dtype], lerr
+    return err, lerr
+
+
+def _w(dtype, B, S, H_q, H_kv, d):
+    base = workloads.WORKLOADS[0 if dtype == torch.float32 else 1]
+    return base.with_(B=B, S=S, H_q=H_q, H_kv=H_kv, d=d)
+
+
+def test_tiny_fp32_workload_full():
+    w = workloads.WORKLOADS[0]
+    inp = workloads.attention_inputs(w, device=DEV)
+    err, lerr = _full_check(inp, torch.float32)
+    print(f"tiny fp32: err/std {err:.2e}, lse {lerr:.2e}")
+
+
+CASES = [
+    # dtype, B, S, H_q, H_kv, d, lens
+    (torch.bfloat16, 3, 16, 32, 8, 128, [0, 1, 300]),
+    (torch.bfloat16, 2, 32, 32, 8, 128, [127, 129]),
+    (torch.bfloat16, 4, 16, 8, 2, 64, [255, 256, 257, 1000]),
+    (torch.bfloat16, 1, 1, 4, 1, 128, [77]),
+    (torch.bfloat16, 2, 64, 4, 2, 64, [10, 515]),
+    (torch.bfloat16, 5, 8, 16, 16, 128, [3, 0, 700, 128, 129]),
+    (torch.float32, 2, 16, 8, 2, 64, [1, 513]),
+    (torch.float32, 3, 32, 8, 2, 128, [0, 0, 0]),
+]
+
+
+@pytest.mark.parametrize("case", CASES)
+def test_small_cases_full(case):
+    dtype, B, S, H_q, H_kv, d, lens = case
+    w = _w(dtype, B, S, H_q, H_kv, d)
+    inp = workloads.attention_inputs(w, device=DEV, lens=lens)
+    _full_check(inp, dtype)
+
+
+def test_explicit_scale_and_padding_rows():
+    w = _w(torch.bfloat16, 3, 16, 16, 4, 128)
+    inp = workloads.attention_inputs(w, device=DEV, lens=[40, 0, 333], pad_rows=13)
+    _full_check(inp, torch.bfloat16, scale=0.05)
+
+
+def test_many_sequences_more_units_than_ctas():
+    w = _w(torch.bfloat16, 300, 16, 8, 2, 64)
+    g = torch.Generator().manual_seed(3)
+    lens = torch.randint(0, 700, (300,), generator=g).tolist()
+    inp = workloads.attention_inputs(w, device=DEV, lens=lens)
+    _full_check(inp, torch.bfloat16)
+
+
+def _sampled_check(inp, dtype, n=48, seed=0):
+    o, lse = _gpu(inp)
+    B, S, H_q, d = inp["q"].shape
+    rng = np.random.default_rng(seed)
+    picks = [(int(rng.integers(B)), int(rng.integers(S)), int(rng.integers(H_q))) for _ in range(n)]
+    picks += [(0, 0, 0), (B - 1, S - 1, H_q - 1)]
+    host = {k: inp[k].cpu() for k in ("q", "k_prefix", "v_prefix", "k_blk", "v_blk")}
+    ro, rl = block_attention_rows(host["q"], host["k_prefix"], host["v_prefix"], host["k_blk"],
+                                  host["v_blk"], inp["prefix_len_host"], inp["prefix_offset_host"],
+                                  picks)
+    og = np.stack([to_np(o[b, i, h]) for (b, i, h) in picks])
+    lg = np.array([float(lse[b, h, i]) for (b, i, h) in picks])
+    sd = to_np(o).std()  # spread of the whole output
+    err = float(np.abs(og - ro).max() / sd)
+    assert err <= ATTN_TOL[dtype], err
+    assert float(np.abs(lg - rl).max()) <= LSE_TOL[dtype]
+    return err
+
+
+@pytest.mark.parametrize("wi", [1, 2, 3])
+def test_full_size_workloads_sampled(wi):
+    w = workloads.WORKLOADS[wi]
+    inp = workloads.attention_inputs(w, device=DEV)
+    err = _sampled_check(inp, torch.bfloat16, n=16 if wi == 3 else 48, seed=wi)
+    print(f"workload {wi}: sampled err/std {err:.2e}")
+
+
+def test_prefix_cache_is_never_written():
+    w = _w(torch.bfloat16, 4, 16, 32, 8, 128)
+    inp = workloads.attention_inputs(w, device=DEV, lens=[500, 20, 0, 1300])
+    before = {k: inp[k].clone() for k in ("k_prefix", "v_prefix", "q", "k_blk", "v_blk")}
+    _gpu(inp)
+    for k, t in before.items():
+        assert torch.equal(t, inp[k]), k
+
+
+def test_device_side_range_error_writes_nothing():
+    w = _w(torch.bfloat16, 2, 16, 8, 2, 64)
+    inp = workloads.attention_inputs(w, device=DEV, lens=[10, 20])
+    inp["prefix_offset"] = torch.tensor([0, 25, 30], dtype=torch.int64, device=DEV)  # 25+20 > 30
+    o = torch.full((2, 16, 8, 64), 7.0, device=DEV)
+    api.attn_step(inp["q"], inp["k_prefix"], inp["v_prefix"], inp["k_blk"], inp["v_blk"],
+                  inp["prefix_len"], inp["prefix_offset"], o=o)
+    assert api.get_device_status() == 5  # BD_ERR_DEVICE_ARG
+    assert bool((o == 7.0).all())
+    assert api.get_device_status() == 0  # cleared by the read
+
+
+def test_permutation_equivariance_on_gpu():
+    w = _w(torch.bfloat16, 2, 16, 32, 8, 128)
+    inp = workloads.attention_inputs(w, device=DEV, lens=[300, 1000])
+    o, _ = _gpu(inp)
+    perm = torch.randperm(16, generator=torch.Generator().manual_seed(5)).to(DEV)
+    pin = dict(inp)
+    for k in ("q", "k_blk", "v_blk"):
+        pin[k] = inp[k][:, perm].contiguous()
+    o2, _ = _gpu(pin)
+    err = float((o2 - o[:, perm]).abs().max() / o.std())
+    assert err < 1e-2, err

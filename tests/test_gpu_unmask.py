@@ -1,0 +1,123 @@
+"""GPU parity of bd_unmask (through the C ABI) against the float64 oracle.
+
+Bar: argmax tokens and commit flags bit-exact, except rows whose top-2 logits
+differ by < 1e-6 (token) or whose confidence is within 1e-6 of gamma (commit),
+which are counted and reported; confidences within 1e-6 absolute.
+"""
+
+import json
+import os
+
+import numpy as np
+import pytest
+import torch
+
+from block_diffusion_lm_bd_b200 import api, workloads
+from oracle.unmask import confidence_unmask
+from _util import compare_unmask
+
+pytestmark = pytest.mark.gpu
+DEV = torch.device("cuda", 0)
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "unmask_small.json")
+
+
+def _run(logits, mask, gamma, block_S=0, fallback=False, **kw):
+    res = api.unmask(logits.to(DEV), mask.to(DEV), gamma, block_S=block_S,
+                     commit_at_least_one=fallback, **kw)
+    torch.cuda.synchronize()
+    assert api.get_device_status() == 0
+    return res
+
+
+def _check(logits, mask, gamma, block_S=0, fallback=False):
+    res = _run(logits, mask, gamma, block_S, fallback, mask_out=torch.empty_like(mask, device=DEV))
+    ref = confidence_unmask(logits.cpu().numpy(), mask.cpu().numpy(), gamma,
+                            block_S=block_S or None, commit_at_least_one=fallback)
+    info = compare_unmask(res, ref, logits.cpu().numpy(), mask, gamma, block_S, fallback)
+    mo = res["mask_out"].cpu().numpy().astype(bool)
+    assert (mo == (mask.cpu().numpy().astype(bool) & ~res["commit"].cpu().numpy().astype(bool))).all()
+    return res, ref, info
+
+
+def test_golden_cases_bit_exact():
+    with open(GOLDEN) as f:
+        cases = json.load(f)["cases"]
+    for c in cases:
+        logits = torch.tensor(c["logits"], dtype=torch.float32)
+        mask = torch.tensor(c["mask"], dtype=torch.uint8)
+        res = _run(logits, mask, c["gamma"], c["block_S"], c["commit_at_least_one"])
+        m = np.asarray(c["mask"]).astype(bool)
+        tok = res["tokens"].cpu().numpy()
+        assert (tok[m] == np.asarray(c["tokens"])[m]).all(), c["name"]
+        assert (tok[~m] == -1).all(), "unmasked rows must be left untouched"
+        assert res["commit"].cpu().numpy().tolist() == c["commit"], c["name"]
+
+
+@pytest.mark.parametrize("wi", [0, 1])
+def test_workload_logits(wi):
+    w = workloads.WORKLOADS[wi]
+    logits = workloads.logits(w, device="cpu")
+    mask = workloads.initial_mask(w)
+    _, ref, info = _check(logits, mask, w.gamma)
+    print(f"workload {wi}: commits {int(ref['commit'].sum())}/{int(mask.sum())}, {info}")
+
+
+def test_loop_step1_size_with_fallback():
+    """B*S = 1024 rows of V = 131072 (the block-loop workload's first step)."""
+    w = workloads.WORKLOADS[4]
+    logits = workloads.logits(w, device="cuda")
+    mask = workloads.initial_mask(w)
+    mask[::3] = 0
+    _check(logits.cpu(), mask, w.gamma, block_S=w.S, fallback=True)
+
+
+def test_ragged_masks_s32():
+    w = workloads.WORKLOADS[2]
+    logits = workloads.logits(w, device="cuda")
+    mask = workloads.initial_mask(w)
+    _check(logits.cpu(), mask, w.gamma)
+
+
+@pytest.mark.parametrize("rows,V", [(1, 1), (3, 3), (5, 7), (17, 1023), (33, 4097), (2, 100003),
+                                    (300, 513), (4096, 64), (16, 131072)])
+def test_odd_sizes_and_alignment(rows, V):
+    g = torch.Generator().manual_seed(rows * 7 + V)
+    logits = torch.randn(rows, V, generator=g) * 2
+    logits[torch.arange(rows), torch.randint(0, V, (rows,), generator=g)] += 9
+    mask = (torch.rand(rows, generator=g) < 0.7).to(torch.uint8)
+    mask[0] = 1
+    _check(logits, mask, 0.5)
+    _check(logits, mask, 0.5, block_S=4, fallback=True)
+
+
+def test_nothing_masked_and_all_ties():
+    logits = torch.zeros(8, 1000)
+    res, _, _ = _check(logits, torch.zeros(8, dtype=torch.uint8), 0.9)
+    assert not res["commit"].any()
+    res, _, _ = _check(logits, torch.ones(8, dtype=torch.uint8), 0.0005)
+    assert (res["tokens"] == 0).all() and res["commit"].all()  # conf = 1/1000 > 0.0005
+
+
+def test_ties_across_segment_boundaries_pick_lowest_index():
+    rows, V = 4, 262144
+    logits = torch.zeros(rows, V)
+    for r, cols in enumerate([(5, 200000), (131071, 131072), (0, V - 1), (99999, 100000, 250000)]):
+        for c in cols:
+            logits[r, c] = 3.0
+    res, _, _ = _check(logits, torch.ones(rows, dtype=torch.uint8), 0.9)
+    assert res["tokens"].cpu().tolist() == [5, 131071, 0, 99999]
+
+
+def test_inplace_mask_update_and_repeat_calls():
+    w = workloads.WORKLOADS[1]
+    logits = workloads.logits(w, device="cuda")
+    mask = torch.ones(logits.shape[0], dtype=torch.uint8, device=DEV)
+    ws = torch.empty(api.unmask_workspace_bytes(*logits.shape), dtype=torch.uint8, device=DEV)
+    ref = confidence_unmask(logits.cpu().numpy(), np.ones(logits.shape[0]), w.gamma)
+    r1 = api.unmask(logits, mask, w.gamma, mask_out="inplace", workspace=ws)
+    n1 = int(mask.sum())
+    assert n1 == int((~ref["commit"]).sum())
+    r2 = api.unmask(logits, mask, w.gamma, mask_out="inplace", workspace=ws)
+    torch.cuda.synchronize()
+    assert int(mask.sum()) == n1  # nothing left passes gamma
+    assert not r2["commit"].any()

@@ -113,3 +113,7 @@ def test_fallback_commits_one_per_unfinished_block():
 def test_top2_gap():
     x = np.array([[1, 3, 3, 0], [0, 5, 1, 2]], dtype=np.float32)
     np.testing.assert_array_equal(top2_gap(x), [0.0, 3.0])
+
+
+def test_top2_gap_single_token_vocabulary():
+    assert np.isinf(top2_gap(np.zeros((3, 1), np.float32))).all()
