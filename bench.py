@@ -1,0 +1,539 @@
+#!/usr/bin/env python
+"""Benchmark of one denoise step (attention over prefix ++ block, then
+confidence unmasking) on B200, printing one JSON line.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
+                    [--workload 1]
+
+Default workload: the bf16 decode step (B=8 sequences, H_q=32, H_kv=8,
+d=128, prefix 4096, block S=16, V=131072, gamma=0.9), synthetic data.
+
+* value: block-tokens/s over all ranks (B*S per step), from CUDA events
+  around K steps replayed as CUDA graphs of library calls, inputs already in
+  HBM, four rotating input sets (> L2) so no step reads another step's data
+  from L2.
+* roofline: the attention call (split-KV kernel + LSE combine) against the
+  measured HBM copy bandwidth; algorithmic bytes = prefix K+V + q + block K/V
+  + o (fp32) + lse.
+* e2e: the same metric through the public API with the step's inputs (q,
+  block K/V, logits, mask) copied from pinned host memory and the unmask
+  result (tokens, confidences, commits) read back every step; the clean-prefix
+  cache is resident state in HBM.
+* cpu_baseline: the float64 oracle on a bounded sample, host cores.
+* --impl reference: the oracle as the reference arm.
+Under torchrun (N > 1) every rank runs an independent replica (replicas
+only: the step has no exchange); the time is the max over ranks.
+"""
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import sys
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import numpy as np
+import torch
+
+PEAKS_FILE = os.path.join(ROOT, "MEASURED_PEAKS.json")
+FALLBACK_HBM = 6650.0
+NOMINAL_HBM = 8000.0
+PROFILE_FILE = os.path.join(ROOT, "profiles", "attn_traffic.json")
+CSRC = os.path.join(ROOT, "block_diffusion_lm_bd_b200", "csrc")
+
+
+def kernel_source_hash():
+    h = hashlib.sha256()
+    for f in sorted(os.listdir(CSRC)):
+        with open(os.path.join(CSRC, f), "rb") as fh:
+            h.update(f.encode() + fh.read())
+    return h.hexdigest()[:16]
+
+
+def hbm_peak():
+    try:
+        with open(PEAKS_FILE) as f:
+            return float(json.load(f)["hbm_gbs"]), "measured"
+    except Exception:
+        return FALLBACK_HBM, "fallback"
+
+
+def dist_env():
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    return world, rank, local
+
+
+def init_dist(world, backend):
+    if world <= 1:
+        return None
+    import datetime
+
+    import torch.distributed as dist
+
+    os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+    dist.init_process_group(backend=backend, timeout=datetime.timedelta(seconds=120))
+    return dist
+
+
+def max_over_ranks(x, dist, device=None):
+    """Max of a float over all ranks (identity without a process group)."""
+    if dist is None:
+        return float(x)
+    t = torch.tensor([float(x)], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def barrier(dist, device=None):
+    if dist is not None:
+        if device is not None and device.type == "cuda":
+            dist.barrier(device_ids=[device.index])
+        else:
+            dist.barrier()
+
+
+# --------------------------------------------------------------------------
+# clocks
+# --------------------------------------------------------------------------
+class ClockSampler:
+    """NVML samples of SM clock and throttle reasons every ~20 ms."""
+
+    REASONS = {
+        "sw_power_cap": 0x4, "hw_slowdown": 0x8, "sw_thermal_slowdown": 0x20,
+        "hw_thermal_slowdown": 0x40, "hw_power_brake_slowdown": 0x80,
+    }
+
+    def __init__(self, device):
+        self.samples, self.reasons, self.ok = [], set(), False
+        self.max_mhz = None
+        self._stop = threading.Event()
+        try:
+            import pynvml
+
+            pynvml.nvmlInit()
+            self.nv = pynvml
+            uuid = str(torch.cuda.get_device_properties(device).uuid)
+            if not uuid.startswith("GPU-"):
+                uuid = "GPU-" + uuid
+            self.h = pynvml.nvmlDeviceGetHandleByUUID(uuid)
+            self.max_mhz = pynvml.nvmlDeviceGetMaxClockInfo(self.h, pynvml.NVML_CLOCK_SM)
+            self.ok = True
+        except Exception:
+            pass
+
+    def _run(self):
+        while not self._stop.is_set():
+            try:
+                self.samples.append(self.nv.nvmlDeviceGetClockInfo(self.h, self.nv.NVML_CLOCK_SM))
+                r = self.nv.nvmlDeviceGetCurrentClocksEventReasons(self.h)
+                for k, bit in self.REASONS.items():
+                    if r & bit:
+                        self.reasons.add(k)
+            except Exception:
+                pass
+            time.sleep(0.02)
+
+    def __enter__(self):
+        if self.ok:
+            self.t = threading.Thread(target=self._run, daemon=True)
+            self.t.start()
+        return self
+
+    def __exit__(self, *a):
+        self._stop.set()
+        if self.ok:
+            self.t.join()
+
+    def summary(self):
+        if not self.samples:
+            return {"sm_mhz": None, "sm_max_mhz": self.max_mhz, "reasons": sorted(self.reasons),
+                    "samples": 0}
+        return {"sm_mhz": statistics.median(self.samples), "sm_max_mhz": self.max_mhz,
+                "reasons": sorted(self.reasons), "samples": len(self.samples)}
+
+
+# --------------------------------------------------------------------------
+# workload
+# --------------------------------------------------------------------------
+def attn_bytes(w, lens):
+    el = 2 if w.dtype == torch.bfloat16 else 4
+    prefix = int(sum(lens)) * w.H_kv * w.d * el * 2
+    q = w.B * w.S * w.H_q * w.d * el
+    blk = 2 * w.B * w.S * w.H_kv * w.d * el
+    o = w.B * w.S * w.H_q * w.d * 4
+    lse = w.B * w.H_q * w.S * 4
+    return prefix + q + blk + o + lse, prefix
+
+
+def unmask_bytes(w, n_masked):
+    return n_masked * w.V * 4 + w.B * w.S * (1 + 4 + 4 + 1)
+
+
+def workload_label(w):
+    return (f"{w.name}: B={w.B} H_q={w.H_q} H_kv={w.H_kv} d={w.d} "
+            f"L={w.prefix_len if w.prefix_range is None else 'U%s' % (w.prefix_range,)} "
+            f"S={w.S} V={w.V} gamma={w.gamma}")
+
+
+def make_sets(w, dev, nsets, rank):
+    from block_diffusion_lm_bd_b200 import workloads
+
+    sets = []
+    for s in range(nsets):
+        inp = workloads.attention_inputs(w, device=dev, step=1000 * rank + s)
+        inp["logits"] = workloads.logits(w, device=dev, step=1000 * rank + s)
+        inp["mask"] = workloads.initial_mask(w).to(dev)
+        sets.append(inp)
+    return sets
+
+
+def run_gpu(args):
+    from block_diffusion_lm_bd_b200 import api, build as _build, workloads
+
+    world, rank, local = dist_env()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    dist = init_dist(world, "nccl")
+    if rank == 0 and _build.needs_build():
+        _build.build()
+    barrier(dist, dev)
+    w = workloads.WORKLOADS[args.workload]
+    nsets = 4
+    sets = make_sets(w, dev, nsets, rank)
+    lens = sets[0]["prefix_len_host"].tolist()
+    B, S, H_q, H_kv, d, V = w.B, w.S, w.H_q, w.H_kv, w.d, w.V
+    rows = B * S
+    ws_a = torch.empty(api.attn_workspace_bytes(B, S, H_q, H_kv, d), dtype=torch.uint8, device=dev)
+    ws_u = torch.empty(api.unmask_workspace_bytes(rows, V), dtype=torch.uint8, device=dev)
+    outs = []
+    for s in range(nsets):
+        outs.append(dict(
+            o=torch.empty((B, S, H_q, d), dtype=torch.float32, device=dev),
+            lse=torch.empty((B, H_q, S), dtype=torch.float32, device=dev),
+            tok=torch.empty(rows, dtype=torch.int32, device=dev),
+            conf=torch.empty(rows, dtype=torch.float32, device=dev),
+            com=torch.empty(rows, dtype=torch.uint8, device=dev),
+        ))
+    stream = torch.cuda.Stream(device=dev)
+
+    def step(i, ev=None):
+        inp, out = sets[i % nsets], outs[i % nsets]
+        if ev is not None:
+            ev[0].record(stream)
+        api.attn_step(inp["q"], inp["k_prefix"], inp["v_prefix"], inp["k_blk"], inp["v_blk"],
+                      inp["prefix_len"], inp["prefix_offset"], o=out["o"], lse=out["lse"],
+                      workspace=ws_a, stream=stream)
+        if ev is not None:
+            ev[1].record(stream)
+        api.unmask(inp["logits"], inp["mask"], w.gamma, block_S=S,
+                   commit_at_least_one=w.commit_at_least_one, tokens_out=out["tok"],
+                   conf_out=out["conf"], commit_out=out["com"], workspace=ws_u, stream=stream)
+        if ev is not None:
+            ev[2].record(stream)
+
+    # eager warm-up (also loads kernels), then graph capture
+    with torch.cuda.stream(stream):
+        for i in range(max(args.warmup, 3)):
+            step(i)
+    stream.synchronize()
+    assert api.get_device_status(stream) == 0
+
+    P = min(args.steps, args.graph_steps)
+    n_full, tail = divmod(args.steps, P)
+    evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)]
+           for _ in range(P)]
+    l0 = api.launch_count()
+    g_main = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_main, stream=stream):
+        for i in range(P):
+            step(i, evs[i])
+    launches_per_step = (api.launch_count() - l0) / P
+    g_tail = None
+    if tail:
+        g_tail = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_tail, stream=stream):
+            for i in range(tail):
+                step(i)
+    # graph warm-up
+    for _ in range(max(1, args.warmup // P)):
+        g_main.replay()
+    torch.cuda.synchronize(dev)
+
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(dev)
+    with sampler:
+        barrier(dist, dev)
+        torch.cuda.synchronize(dev)
+        with torch.cuda.stream(stream):
+            t0.record(stream)
+            for _ in range(n_full):
+                g_main.replay()
+            if g_tail is not None:
+                g_tail.replay()
+            t1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(dist, dev)
+    st = api.get_device_status(stream)
+    if st != 0:
+        raise RuntimeError(f"device status {api.status_string(st)}")
+    ms_local = t0.elapsed_time(t1)
+    ms = max_over_ranks(ms_local, dist, dev)
+    attn_ms = [e[0].elapsed_time(e[1]) for e in evs]
+    um_ms = [e[1].elapsed_time(e[2]) for e in evs]
+    attn_avg_ms = max_over_ranks(sum(attn_ms) / len(attn_ms), dist, dev)
+    um_avg_ms = max_over_ranks(sum(um_ms) / len(um_ms), dist, dev)
+
+    # e2e: public API with host buffers
+    e2e = run_e2e(args, w, sets, outs, ws_a, ws_u, stream, dev, dist)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        cpu = run_cpu_baseline(w, args.cpu_seconds)
+
+    if rank == 0:
+        peak, peak_kind = hbm_peak()
+        abytes, prefix_bytes = attn_bytes(w, lens)
+        n_masked = int(sets[0]["mask"].sum())
+        ubytes = unmask_bytes(w, n_masked)
+        units = rows * args.steps * world
+        achieved = abytes / (attn_avg_ms * 1e-3) / 1e9
+        traffic = load_traffic(w)
+        rec = {
+            "metric": "denoise-step block-tokens/s",
+            "value": units / (ms * 1e-3),
+            "unit": "block-tokens/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": ms / args.steps,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16" if w.dtype == torch.bfloat16 else "f32",
+            "data": "synthetic (seeded; shapes of the pages' workloads)",
+            "config": {
+                "workload": workload_label(w),
+                "B": B, "S": S, "H_q": H_q, "H_kv": H_kv, "d": d, "prefix_tokens": int(sum(lens)),
+                "V": V, "gamma": w.gamma, "masked_rows": n_masked,
+                "l2": f"{nsets} rotating input sets of "
+                      f"{(abytes + ubytes) / 1e6:.0f} MB each (> 126 MB L2)",
+                "timing": f"CUDA graphs of {P} steps of library calls, CUDA events",
+                "parallelism": f"replicas x{world}",
+            },
+            "roofline": {
+                "bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                "frac": achieved / peak, "traffic": traffic,
+                "peak_kind": peak_kind, "frac_of_nominal_8000": achieved / NOMINAL_HBM,
+                "kernel": "bd_attn_step (split-KV attention + LSE combine)",
+                "algorithmic_bytes": abytes, "prefix_kv_bytes": prefix_bytes,
+                "avg_call_us": attn_avg_ms * 1e3,
+                "prefix_kv_gbs": prefix_bytes / (attn_avg_ms * 1e-3) / 1e9,
+            },
+            "roofline_unmask": {
+                "bound": "hbm", "achieved": ubytes / (um_avg_ms * 1e-3) / 1e9, "peak": peak,
+                "unit": "GB/s", "frac": ubytes / (um_avg_ms * 1e-3) / 1e9 / peak,
+                "algorithmic_bytes": ubytes, "avg_call_us": um_avg_ms * 1e3,
+            },
+            "gpu_launches": int(round(launches_per_step * args.steps)),
+            "clocks": sampler.summary(),
+            "e2e": e2e,
+            "cpu_baseline": cpu,
+            "kernel_source": kernel_source_hash(),
+        }
+        print(json.dumps(rec))
+    if dist is not None:
+        dist.destroy_process_group()
+
+
+def run_e2e(args, w, sets, outs, ws_a, ws_u, stream, dev, dist):
+    from block_diffusion_lm_bd_b200 import api
+
+    nsets = len(sets)
+    keys_in = ["q", "k_blk", "v_blk", "logits", "mask"]
+    host = [{k: sets[s][k].to("cpu").pin_memory() for k in keys_in} for s in range(nsets)]
+    res_host = [{k: torch.empty(outs[s][k].shape, dtype=outs[s][k].dtype).pin_memory()
+                 for k in ("tok", "conf", "com")} for s in range(nsets)]
+    h2d = sum(t.numel() * t.element_size() for t in host[0].values())
+    d2h = sum(t.numel() * t.element_size() for t in res_host[0].values())
+    K = min(args.steps, args.e2e_steps)
+
+    def e2e_step(i):
+        s = i % nsets
+        inp, out = sets[s], outs[s]
+        for k in keys_in:
+            inp[k].copy_(host[s][k], non_blocking=True)
+        api.attn_step(inp["q"], inp["k_prefix"], inp["v_prefix"], inp["k_blk"], inp["v_blk"],
+                      inp["prefix_len"], inp["prefix_offset"], o=out["o"], lse=out["lse"],
+                      workspace=ws_a, stream=stream)
+        api.unmask(inp["logits"], inp["mask"], w.gamma, block_S=w.S,
+                   commit_at_least_one=w.commit_at_least_one, tokens_out=out["tok"],
+                   conf_out=out["conf"], commit_out=out["com"], workspace=ws_u, stream=stream)
+        for k in ("tok", "conf", "com"):
+            res_host[s][k].copy_(out[k], non_blocking=True)
+
+    with torch.cuda.stream(stream):
+        for i in range(3):
+            e2e_step(i)
+        stream.synchronize()
+        barrier(dist, dev)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        for i in range(K):
+            e2e_step(i)
+        b.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(dist, dev)
+    ms = max_over_ranks(a.elapsed_time(b), dist, dev)
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    return {"value": w.B * w.S * K * world / (ms * 1e-3), "unit": "block-tokens/s",
+            "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": K,
+            "ms_per_step": ms / K}
+
+
+def load_traffic(w):
+    """DRAM bytes per attention call from the committed ncu summary, if the
+    kernel sources are unchanged since it was taken (else None)."""
+    try:
+        with open(PROFILE_FILE) as f:
+            prof = json.load(f)
+        if prof.get("kernel_source") != kernel_source_hash():
+            return None
+        return prof.get("traffic_per_call", {}).get(str(w.index))
+    except Exception:
+        return None
+
+
+# --------------------------------------------------------------------------
+# CPU: the oracle
+# --------------------------------------------------------------------------
+def oracle_unit_inputs(w, seq=0):
+    """Host inputs of one sequence of the workload, for the oracle."""
+    from block_diffusion_lm_bd_b200 import workloads
+
+    L = int(workloads.prefix_lengths(w)[seq])
+    one = w.with_(B=1, prefix_range=None, prefix_len=L)
+    inp = workloads.attention_inputs(one, device="cpu", step=seq)
+    logits = workloads.logits(one, device="cpu", step=seq)
+    mask = workloads.initial_mask(one)
+    return one, inp, logits, mask
+
+
+def oracle_unit(one, inp, logits, mask, kv):
+    """The oracle on 1/H_kv of one sequence's step: the g query heads of KV
+    head kv over prefix + block keys, and S/H_kv of the unmask rows."""
+    from oracle.attention import block_attention
+    from oracle.unmask import confidence_unmask
+
+    g = one.g
+    block_attention(inp["q"][:, :, kv * g:(kv + 1) * g], inp["k_prefix"][:, kv:kv + 1],
+                    inp["v_prefix"][:, kv:kv + 1], inp["k_blk"][:, :, kv:kv + 1],
+                    inp["v_blk"][:, :, kv:kv + 1], inp["prefix_len_host"],
+                    inp["prefix_offset_host"])
+    r = max(1, one.S // one.H_kv)
+    lo = (kv * r) % one.S
+    confidence_unmask(logits[lo:lo + r].numpy(), mask[lo:lo + r].numpy(), one.gamma)
+    return one.S / one.H_kv  # block-tokens' worth of work
+
+
+def cpu_threads():
+    try:
+        from threadpoolctl import threadpool_info
+
+        n = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:
+        n = 1
+    return n
+
+
+def _unit_sample_text(w):
+    return (f"one KV-head group of one sequence per unit ({w.g} query heads x {w.S} block "
+            f"positions over its prefix + {w.S} block keys) and {max(1, w.S // w.H_kv)} unmask "
+            f"rows of {w.V} logits = 1/{w.H_kv} of one sequence's step, float64 NumPy")
+
+
+def run_cpu_baseline(w, seconds):
+    cache = [oracle_unit_inputs(w, s) for s in range(min(w.B, 2))]
+    tokens, t, n = 0.0, 0.0, 0
+    while t < seconds:
+        one, inp, logits, mask = cache[n % len(cache)]
+        t0 = time.perf_counter()
+        tokens += oracle_unit(one, inp, logits, mask, n % one.H_kv)
+        t += time.perf_counter() - t0
+        n += 1
+    return {"value": tokens / t, "unit": "block-tokens/s", "cores": cpu_threads(), "kind": "oracle",
+            "sample": f"{n} units in {t:.1f} s; " + _unit_sample_text(w),
+            "host_cpus": len(os.sched_getaffinity(0))}
+
+
+def run_reference(args):
+    world, rank, _ = dist_env()
+    if rank != 0:
+        return
+    from block_diffusion_lm_bd_b200 import workloads
+
+    w = workloads.WORKLOADS[args.workload]
+    cache = [oracle_unit_inputs(w, s) for s in range(min(w.B, 2))]
+    for i in range(args.warmup):
+        oracle_unit(*cache[i % len(cache)], i % w.H_kv)
+    tokens, t = 0.0, 0.0
+    for i in range(args.steps):
+        one, inp, logits, mask = cache[i % len(cache)]
+        t0 = time.perf_counter()
+        tokens += oracle_unit(one, inp, logits, mask, i % w.H_kv)
+        t += time.perf_counter() - t0
+    value = tokens / t
+    rec = {
+        "impl": "reference",
+        "metric": "denoise-step block-tokens/s",
+        "value": value,
+        "unit": "block-tokens/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": t / args.steps * 1e3,
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "f64",
+        "data": "synthetic (seeded; shapes of the pages' workloads)",
+        "config": {"workload": workload_label(w), "parallelism": "host cores"},
+        "cpu_baseline": {"value": value, "unit": "block-tokens/s", "cores": cpu_threads(),
+                         "kind": "oracle", "sample": "each step: " + _unit_sample_text(w)},
+        "e2e": {"value": value, "unit": "block-tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(rec))
+
+
+def main(argv=None):
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=4000)
+    ap.add_argument("--warmup", type=int, default=50)
+    ap.add_argument("--impl", default="native", choices=["native", "reference"])
+    ap.add_argument("--workload", type=int, default=1, choices=[1, 2, 3])
+    ap.add_argument("--graph-steps", type=int, default=400)
+    ap.add_argument("--e2e-steps", type=int, default=200)
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args(argv)
+    if args.warmup < 3:
+        args.warmup = 3
+    if args.impl == "reference":
+        run_reference(args)
+    else:
+        run_gpu(args)
+
+
+if __name__ == "__main__":
+    main()

@@ -23,7 +23,6 @@ namespace bd {
 constexpr int kUnitKeys = 128;     // prefix keys per work unit
 constexpr int kMaxBatch = 4096;    // sequences per call
 constexpr int kMaxRows = 128;      // packed query rows g*S per (b, kv)
-constexpr int kPlanThreads = 256;  // scan width of the in-kernel plan
 
 struct AttnWs {
   int *flag;     // [1]  1: device-side argument error, nothing was written
@@ -76,32 +75,33 @@ struct PlanStart {
   bool bad;     // some prefix_len / prefix_offset is out of range
 };
 
-// Block-wide plan: every thread of the CTA must call it. `e0` is the CTA's
-// first unit, computed from W inside (so passed as the CTA index).
+// Block-wide plan: every thread of the CTA must call it; s_scan holds
+// blockDim.x ints. The CTA's first unit is start(cta) of the partition of W.
 __device__ inline PlanStart attn_plan(const AttnParams &p, int cta, int *s_scan, int *s_misc) {
   const int tid = threadIdx.x;
+  const int nt = blockDim.x;
   // pass 1: total units and range check
   int carry = 0;
   int bad = 0;
-  for (int base = 0; base < p.B; base += kPlanThreads) {
+  for (int base = 0; base < p.B; base += nt) {
     const int b = base + tid;
     int n = 0;
-    if (b < p.B && tid < kPlanThreads) {
+    if (b < p.B && tid < nt) {
       const int L = p.prefix_len[b];
       const int64_t off = p.prefix_offset[b];
       if (L < 0 || off < 0 || off + L > p.prefix_rows) bad = 1;
       n = attn_units(L < 0 ? 0 : L);
     }
-    if (tid < kPlanThreads) s_scan[tid] = n;
+    if (tid < nt) s_scan[tid] = n;
     __syncthreads();
-    for (int o = 1; o < kPlanThreads; o <<= 1) {
-      int v = (tid < kPlanThreads && tid >= o) ? s_scan[tid - o] : 0;
+    for (int o = 1; o < nt; o <<= 1) {
+      int v = (tid < nt && tid >= o) ? s_scan[tid - o] : 0;
       __syncthreads();
-      if (tid < kPlanThreads) s_scan[tid] += v;
+      if (tid < nt) s_scan[tid] += v;
       __syncthreads();
     }
-    if (cta == 0 && b < p.B && tid < kPlanThreads) p.ws.cum[b] = carry + s_scan[tid] - n;
-    carry += s_scan[kPlanThreads - 1];
+    if (cta == 0 && b < p.B && tid < nt) p.ws.cum[b] = carry + s_scan[tid] - n;
+    carry += s_scan[nt - 1];
     __syncthreads();
   }
   if (tid == 0) s_misc[0] = 0;
@@ -126,26 +126,26 @@ __device__ inline PlanStart attn_plan(const AttnParams &p, int cta, int *s_scan,
   }
   carry = 0;
   __syncthreads();
-  for (int base = 0; base < p.B; base += kPlanThreads) {
+  for (int base = 0; base < p.B; base += nt) {
     const int b = base + tid;
     int n = 0;
-    if (b < p.B && tid < kPlanThreads) n = attn_units(max(0, p.prefix_len[b]));
-    if (tid < kPlanThreads) s_scan[tid] = n;
+    if (b < p.B && tid < nt) n = attn_units(max(0, p.prefix_len[b]));
+    if (tid < nt) s_scan[tid] = n;
     __syncthreads();
-    for (int o = 1; o < kPlanThreads; o <<= 1) {
-      int v = (tid < kPlanThreads && tid >= o) ? s_scan[tid - o] : 0;
+    for (int o = 1; o < nt; o <<= 1) {
+      int v = (tid < nt && tid >= o) ? s_scan[tid - o] : 0;
       __syncthreads();
-      if (tid < kPlanThreads) s_scan[tid] += v;
+      if (tid < nt) s_scan[tid] += v;
       __syncthreads();
     }
-    if (b < p.B && tid < kPlanThreads) {
+    if (b < p.B && tid < nt) {
       const int ex = carry + s_scan[tid] - n;
       if (int64_t(p.H_kv) * ex <= e0 && e0 < int64_t(p.H_kv) * (ex + n)) {
         s_misc[1] = b;
         s_misc[2] = ex;
       }
     }
-    carry += s_scan[kPlanThreads - 1];
+    carry += s_scan[nt - 1];
     __syncthreads();
   }
   ps.b = s_misc[1];
@@ -153,6 +153,56 @@ __device__ inline PlanStart attn_plan(const AttnParams &p, int cta, int *s_scan,
   __syncthreads();
   return ps;
 }
+
+// Walks a CTA's range of units segment by segment (one segment = the units of
+// one (b, kv) pair inside the range). Every role of a CTA runs its own copy.
+struct SegWalker {
+  int64_t e, e0, e1;
+  int b, kv, cum_b, L, n;
+  int64_t off;
+  // the segment returned by the last next()
+  int sb, skv, sL, sn, u0, u1;
+  int64_t soff;
+  bool first, complete;
+
+  __device__ void init(const AttnParams &p, const PlanStart &ps, int64_t e0_, int64_t e1_) {
+    e0 = e0_;
+    e1 = e1_;
+    e = e0_;
+    b = ps.b;
+    cum_b = ps.cum_b;
+    L = p.prefix_len[b];
+    off = p.prefix_offset[b];
+    n = attn_units(L);
+    kv = int((e0 - int64_t(p.H_kv) * cum_b) / n);
+  }
+
+  __device__ bool next(const AttnParams &p) {
+    if (e >= e1) return false;
+    const int64_t pbase = int64_t(p.H_kv) * cum_b + int64_t(kv) * n;
+    u0 = int(e - pbase);
+    u1 = int(e1 - pbase < int64_t(n) ? e1 - pbase : int64_t(n));
+    first = (e == e0);
+    complete = (u0 == 0 && u1 == n);
+    sb = b;
+    skv = kv;
+    sL = L;
+    sn = n;
+    soff = off;
+    e = pbase + u1;
+    if (++kv == p.H_kv) {
+      kv = 0;
+      cum_b += n;
+      ++b;
+      if (b < p.B) {
+        L = p.prefix_len[b];
+        off = p.prefix_offset[b];
+        n = attn_units(L);
+      }
+    }
+    return true;
+  }
+};
 
 // Index of the boundary slot a segment writes to.
 __device__ __forceinline__ int64_t attn_slot_index(int cta, bool first) {

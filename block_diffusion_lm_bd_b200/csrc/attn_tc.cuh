@@ -1,0 +1,505 @@
+// Split-KV attention of the active block on the sm_100a tensor cores.
+//
+// "Technical summary: Nemotron-TwoTower", Methodology > Architecture item 2 and
+// Generation process third bullet: each block query attends to the clean-prefix
+// KV of the context tower and to the block's own KV in one softmax. Here the
+// g = H_q / H_kv query heads of a KV head times the S block positions are packed
+// into one M = g*S <= 128 row tile, so every prefix K/V byte is read from HBM
+// once per KV head.
+//
+// One persistent CTA per SM walks its balanced range of work units
+// (attn_common.cuh). Warp roles (192 threads):
+//   warp 0      TMA producer: Q tile per segment, then K and V tiles of
+//               128 keys (2 x 64-column 128B-swizzled panels each) into a
+//               3-stage shared-memory ring.
+//   warp 1      MMA issuer (one thread): S = Q K^T into a double-buffered TMEM
+//               score tile (tcgen05.mma, A and B from shared memory), then
+//               O += P V with P read from TMEM and V from shared memory
+//               (MN-major descriptor). Also owns the TMEM allocation.
+//   warps 2-5   softmax / epilogue, one TMEM lane (= one query row) per
+//               thread: base-2 online softmax with a lazy maximum (O is
+//               rescaled only when a row maximum grows by more than 2^8),
+//               P written back over the score columns as bf16, and at the
+//               end of a segment O / l written to o (or to a boundary slot).
+// Every mbarrier wait is bounded; a wait that runs out records
+// BD_ERR_TIMEOUT, raises a CTA-wide abort flag and the CTA drains its
+// outstanding copies / MMAs (bounded) before releasing TMEM and exiting.
+#pragma once
+
+#include "attn_common.cuh"
+#include "tc_ptx.cuh"
+
+namespace bd {
+
+constexpr int kTcThreads = 192;
+constexpr int kTcStages = 3;
+constexpr int kTcKeys = 128;                       // keys per tile (= kUnitKeys)
+constexpr uint32_t kPanelBytes = 128 * 128;        // 128 rows x 128 B
+constexpr uint32_t kTileBytes = 2 * kPanelBytes;   // 128 x 128 bf16
+constexpr uint32_t kStageBytes = 2 * kTileBytes;   // K + V
+constexpr uint32_t kTmemCols = 512;
+constexpr uint32_t kTmemO = 0;                     // O accumulator columns [0,128)
+constexpr uint32_t kTmemS = 128;                   // score buffer b at 128 + 128 b
+
+// dynamic shared memory layout (offsets from a 1024-byte aligned base)
+constexpr uint32_t kSmQ = 0;
+constexpr uint32_t kSmStage = kTileBytes;
+constexpr uint32_t kSmBar = kSmStage + kTcStages * kStageBytes;
+// barriers: kv_full[S], kv_empty[S], q_full, q_empty, s_full[2], p_full[2], o_ready, o_free,
+//           mma_done
+constexpr int kNumBars = 2 * kTcStages + 9;
+constexpr uint32_t kSmTmemSlot = kSmBar + 8 * kNumBars;
+constexpr uint32_t kSmAbort = kSmTmemSlot + 8;
+constexpr uint32_t kSmEnd = kSmAbort + 8;
+constexpr size_t kTcSmemBytes = kSmEnd + 1024;  // + alignment slack
+
+static_assert(kTcKeys == kUnitKeys, "one tensor-core tile per work unit");
+
+struct TcBars {
+  uint32_t kv_full, kv_empty, q_full, q_empty, s_full, p_full, o_ready, o_free, mma_done;
+  __device__ TcBars(uint32_t base) {
+    kv_full = base;
+    kv_empty = base + 8 * kTcStages;
+    q_full = base + 16 * kTcStages;
+    q_empty = q_full + 8;
+    s_full = q_full + 16;  // [2]
+    p_full = q_full + 32;  // [2]
+    o_ready = q_full + 48;
+    o_free = q_full + 56;
+    mma_done = q_full + 64;
+  }
+};
+
+__device__ __forceinline__ bool tc_wait(uint32_t bar, uint32_t phase, uint32_t max_polls,
+                                        volatile int *abort_flag) {
+  uint32_t ok;
+  for (uint32_t i = 0;; ++i) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+        "selp.u32 %0, 1, 0, p;\n\t}"
+        : "=r"(ok)
+        : "r"(bar), "r"(phase)
+        : "memory");
+    if (ok) return true;
+    if ((i & 255) == 255 && *abort_flag) return false;
+    if (i >= max_polls) {
+      record_status(BD_ERR_TIMEOUT);
+      *abort_flag = 1;
+      return false;
+    }
+    if (i > 256) __nanosleep(64);
+  }
+}
+
+__device__ __forceinline__ void bar_init(uint32_t bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(bar), "r"(count));
+}
+__device__ __forceinline__ void bar_arrive(uint32_t bar) {
+  asm volatile("{\n\t.reg .b64 st;\n\tmbarrier.arrive.shared::cta.b64 st, [%0];\n\t}" ::"r"(bar)
+               : "memory");
+}
+__device__ __forceinline__ void bar_expect_tx(uint32_t bar, uint32_t bytes) {
+  asm volatile(
+      "{\n\t.reg .b64 st;\n\tmbarrier.arrive.expect_tx.shared::cta.b64 st, [%0], %1;\n\t}" ::"r"(
+          bar),
+      "r"(bytes)
+      : "memory");
+}
+
+__global__ void __launch_bounds__(kTcThreads, 1)
+    attn_tc_kernel(const __grid_constant__ CUtensorMap tm_q, const __grid_constant__ CUtensorMap tm_kp,
+                   const __grid_constant__ CUtensorMap tm_vp, const __grid_constant__ CUtensorMap tm_kb,
+                   const __grid_constant__ CUtensorMap tm_vb, const AttnParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  __shared__ int s_scan[kTcThreads];
+  __shared__ int s_misc[4];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;
+  uint8_t *smem = smem_raw + (sbase - raw);
+  const TcBars bars(sbase + kSmBar);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kSmTmemSlot);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kSmAbort);
+
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int cta = blockIdx.x;
+  const PlanStart ps = attn_plan(p, cta, s_scan, s_misc);
+  pdl_launch_dependents();
+  if (ps.bad) {
+    if (cta == 0 && tid == 0) record_status(BD_ERR_DEVICE_ARG);
+    return;
+  }
+  if (ps.W == 0) return;
+  const int64_t e0 = part_start(cta, ps.W, p.G), e1 = part_start(cta + 1, ps.W, p.G);
+  if (e1 <= e0) return;
+
+  if (tid == 0) {
+    for (int i = 0; i < kTcStages; ++i) {
+      bar_init(bars.kv_full + 8 * i, 1);
+      bar_init(bars.kv_empty + 8 * i, 1);
+    }
+    bar_init(bars.q_full, 1);
+    bar_init(bars.q_empty, 1);
+    for (int i = 0; i < 2; ++i) {
+      bar_init(bars.s_full + 8 * i, 1);
+      bar_init(bars.p_full + 8 * i, 4);
+    }
+    bar_init(bars.o_ready, 1);
+    bar_init(bars.o_free, 4);
+    bar_init(bars.mma_done, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    prefetch_tmap(&tm_q);
+    prefetch_tmap(&tm_kp);
+    prefetch_tmap(&tm_vp);
+    prefetch_tmap(&tm_kb);
+    prefetch_tmap(&tm_vb);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  SegWalker wk;
+  wk.init(p, ps, e0, e1);
+  const uint32_t mp = p.max_polls;
+  const int S16 = (p.S + 15) & ~15;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      uint32_t t = 0;
+      int seg = 0;
+      bool ok = true;
+      const uint32_t q_bytes = 2u * 128u * uint32_t(p.M);
+      const uint32_t blk_bytes = 4u * 128u * uint32_t(S16);
+      while (ok && wk.next(p)) {
+        if (seg > 0 && !tc_wait(bars.q_empty, (seg - 1) & 1, mp, abort_flag)) {
+          ok = false;
+          break;
+        }
+        bar_expect_tx(bars.q_full, q_bytes);
+        tma_load_3d(sbase + kSmQ, &tm_q, bars.q_full, 0, wk.skv * p.g, wk.sb * p.S);
+        tma_load_3d(sbase + kSmQ + kPanelBytes, &tm_q, bars.q_full, 64, wk.skv * p.g,
+                    wk.sb * p.S);
+        for (int u = wk.u0; u < wk.u1; ++u, ++t) {
+          const uint32_t st = t % kTcStages;
+          if (t >= kTcStages &&
+              !tc_wait(bars.kv_empty + 8 * st, ((t / kTcStages) - 1) & 1, mp, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const uint32_t kdst = sbase + kSmStage + st * kStageBytes;
+          const uint32_t vdst = kdst + kTileBytes;
+          const uint32_t fb = bars.kv_full + 8 * st;
+          if (u < wk.sn - 1) {
+            const int z = int(wk.soff + int64_t(u) * kTcKeys);
+            bar_expect_tx(fb, 4 * kPanelBytes);
+            tma_load_3d(kdst, &tm_kp, fb, 0, wk.skv, z);
+            tma_load_3d(kdst + kPanelBytes, &tm_kp, fb, 64, wk.skv, z);
+            tma_load_3d(vdst, &tm_vp, fb, 0, wk.skv, z);
+            tma_load_3d(vdst + kPanelBytes, &tm_vp, fb, 64, wk.skv, z);
+          } else {
+            const int z = wk.sb * p.S;
+            bar_expect_tx(fb, blk_bytes);
+            tma_load_3d(kdst, &tm_kb, fb, 0, wk.skv, z);
+            tma_load_3d(kdst + kPanelBytes, &tm_kb, fb, 64, wk.skv, z);
+            tma_load_3d(vdst, &tm_vb, fb, 0, wk.skv, z);
+            tma_load_3d(vdst + kPanelBytes, &tm_vb, fb, 64, wk.skv, z);
+          }
+        }
+        ++seg;
+      }
+      if (!ok) {
+        // drain: the newest load of each stage and the newest Q load must land
+        // before the CTA may exit
+        for (uint32_t k = 0; k < kTcStages && k < t; ++k) {
+          const uint32_t tl = t - 1 - k;
+          tc_wait(bars.kv_full + 8 * (tl % kTcStages), (tl / kTcStages) & 1, mp, abort_flag);
+        }
+        if (seg > 0) tc_wait(bars.q_full, (seg - 1) & 1, mp, abort_flag);
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      const uint32_t id_qk = idesc_bf16(128, kTcKeys, 0);
+      const uint32_t id_qb = idesc_bf16(128, S16, 0);
+      const uint32_t id_pv = idesc_bf16(128, 128, 1);
+      uint32_t t = 0;
+      int seg = 0;
+      bool ok = true;
+      // P.V of tile tp (its P is in score buffer tp & 1, its V in stage tp % S)
+      auto issue_pv = [&](uint32_t tp, int nkeys, bool first_pv) -> bool {
+        if (first_pv && seg > 0 && !tc_wait(bars.o_free, (seg - 1) & 1, mp, abort_flag))
+          return false;
+        if (!tc_wait(bars.p_full + 8 * (tp & 1), (tp >> 1) & 1, mp, abort_flag)) return false;
+        tc_fence_after();
+        const uint32_t vsm = sbase + kSmStage + (tp % kTcStages) * kStageBytes + kTileBytes;
+        const uint32_t pcol = tmem + kTmemS + 128u * (tp & 1);
+        for (int k = 0; k < nkeys / 16; ++k) {
+          const uint64_t bd = sdesc_sw128(vsm + uint32_t(k) * 2048u, kPanelBytes, 1024);
+          mma_ts(tmem + kTmemO, pcol + uint32_t(k) * 8u, bd, id_pv, (first_pv && k == 0) ? 0u : 1u);
+        }
+        tc_commit(bars.kv_empty + 8 * (tp % kTcStages));
+        tc_commit(bars.o_ready);
+        return true;
+      };
+      while (ok && wk.next(p)) {
+        if (!tc_wait(bars.q_full, seg & 1, mp, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const int nt = wk.u1 - wk.u0;
+        int nprev = 0;
+        for (int i = 0; i < nt; ++i, ++t) {
+          const int u = wk.u0 + i;
+          const uint32_t st = t % kTcStages, sb = t & 1;
+          if (!tc_wait(bars.kv_full + 8 * st, (t / kTcStages) & 1, mp, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const bool blk = (u == wk.sn - 1);
+          const uint32_t ksm = sbase + kSmStage + st * kStageBytes;
+          const uint32_t dcol = tmem + kTmemS + 128u * sb;
+#pragma unroll
+          for (int k = 0; k < 8; ++k) {
+            const uint32_t off = uint32_t(k >> 2) * kPanelBytes + uint32_t(k & 3) * 32u;
+            const uint64_t ad = sdesc_sw128(sbase + kSmQ + off, 16, 1024);
+            const uint64_t bd = sdesc_sw128(ksm + off, 16, 1024);
+            mma_ss(dcol, ad, bd, blk ? id_qb : id_qk, k > 0 ? 1u : 0u);
+          }
+          tc_commit(bars.s_full + 8 * sb);
+          if (i == nt - 1) tc_commit(bars.q_empty);
+          if (i > 0 && !issue_pv(t - 1, nprev, i == 1)) {
+            ok = false;
+            break;
+          }
+          nprev = blk ? S16 : kTcKeys;
+        }
+        if (!ok) break;
+        if (!issue_pv(t - 1, nprev, nt == 1)) {
+          ok = false;
+          break;
+        }
+        ++seg;
+      }
+      if (!ok) {
+        tc_commit(bars.mma_done);
+        tc_wait(bars.mma_done, 0, mp, abort_flag);
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ softmax / epilogue
+    const int q4 = warp & 3;
+    const int row = q4 * 32 + lane;
+    const bool active = q4 * 32 < p.M;  // warp-uniform
+    const uint32_t lrow = uint32_t(q4 * 32) << 16;
+    const float c2 = p.scale_log2;
+    uint32_t t = 0;
+    bool ok = true;
+    while (ok && wk.next(p)) {
+      float m_run = -INFINITY, l_run = 0.f;
+      const int nt = wk.u1 - wk.u0;
+      for (int i = 0; i < nt; ++i, ++t) {
+        const int u = wk.u0 + i;
+        const uint32_t sb = t & 1;
+        if (!__all_sync(0xffffffffu, tc_wait(bars.s_full + 8 * sb, (t >> 1) & 1, mp, abort_flag))) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        const bool blk = (u == wk.sn - 1);
+        const int nvalid = blk ? p.S : min(kTcKeys, wk.sL - u * kTcKeys);
+        float alpha = 1.f;
+        bool resc = false;
+        if (active) {
+          const uint32_t sc = tmem + lrow + kTmemS + 128u * sb;
+          float x[128];
+#pragma unroll
+          for (int c0 = 0; c0 < 128; c0 += 32) {
+            uint32_t r[32];
+            tmem_ld_x32(sc + c0, r);
+#pragma unroll
+            for (int j = 0; j < 32; ++j) x[c0 + j] = __uint_as_float(r[j]);
+          }
+          float mt = -INFINITY;
+#pragma unroll
+          for (int c = 0; c < 128; ++c) {
+            x[c] = (c < nvalid) ? x[c] * c2 : -INFINITY;
+            mt = fmaxf(mt, x[c]);
+          }
+          if (i == 0) {
+            m_run = mt;
+          } else if (mt > m_run + 8.f) {
+            alpha = exp2f(m_run - mt);
+            l_run *= alpha;
+            m_run = mt;
+            resc = true;
+          }
+          float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+          for (int c0 = 0; c0 < 128; c0 += 64) {
+            uint32_t pk[32];
+#pragma unroll
+            for (int j = 0; j < 32; ++j) {
+              const float a = exp2f(x[c0 + 2 * j] - m_run);
+              const float b = exp2f(x[c0 + 2 * j + 1] - m_run);
+              s0 += a;
+              s1 += b;
+              pk[j] = pack_bf16x2(a, b);
+            }
+            tmem_st_x32(sc + uint32_t(c0 / 2), pk);
+          }
+          l_run += s0 + s1;
+        }
+        if (i > 0) {
+          // P.V of the previous tile must be complete before O may be rescaled
+          // and before the next P.V is released
+          if (!__all_sync(0xffffffffu, tc_wait(bars.o_ready, (t - 1) & 1, mp, abort_flag))) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          if (active && __any_sync(0xffffffffu, resc)) {
+            const uint32_t oc = tmem + lrow + kTmemO;
+#pragma unroll
+            for (int c0 = 0; c0 < 128; c0 += 32) {
+              uint32_t r[32];
+              tmem_ld_x32(oc + c0, r);
+#pragma unroll
+              for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(__uint_as_float(r[j]) * alpha);
+              tmem_st_x32(oc + c0, r);
+            }
+          }
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) bar_arrive(bars.p_full + 8 * sb);
+      }
+      if (!ok) break;
+      // epilogue: O / l of this segment
+      if (!__all_sync(0xffffffffu, tc_wait(bars.o_ready, (t - 1) & 1, mp, abort_flag))) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      if (active) {
+        // loads are warp-wide (.sync.aligned); only rows < M store
+        const bool live = row < p.M;
+        const int m = live ? row : 0;
+        const int s = m / p.g, j = m % p.g;
+        const float inv = 1.f / l_run;
+        const float lse = (m_run + log2f(l_run)) * 0.69314718055994531f;
+        float *dst;
+        if (wk.complete) {
+          dst = p.o + ((int64_t(wk.sb) * p.S + s) * p.H_q + wk.skv * p.g + j) * 128;
+          if (live && p.lse) p.lse[(int64_t(wk.sb) * p.H_q + wk.skv * p.g + j) * p.S + s] = lse;
+        } else {
+          const int64_t slot = attn_slot_index(cta, wk.first);
+          dst = p.ws.slot + (slot * p.M + m) * 128;
+          if (live) p.ws.slot_lse[slot * p.M + m] = lse;
+        }
+        const uint32_t oc = tmem + lrow + kTmemO;
+#pragma unroll
+        for (int c0 = 0; c0 < 128; c0 += 32) {
+          uint32_t r[32];
+          tmem_ld_x32(oc + c0, r);
+          if (live) {
+#pragma unroll
+            for (int j4 = 0; j4 < 8; ++j4) {
+              const float4 v = make_float4(
+                  __uint_as_float(r[4 * j4]) * inv, __uint_as_float(r[4 * j4 + 1]) * inv,
+                  __uint_as_float(r[4 * j4 + 2]) * inv, __uint_as_float(r[4 * j4 + 3]) * inv);
+              *reinterpret_cast<float4 *>(dst + c0 + 4 * j4) = v;
+            }
+          }
+        }
+      }
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) bar_arrive(bars.o_free);
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, kTmemCols);
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+typedef CUresult (*EncodeTiledFn)(CUtensorMap *, CUtensorMapDataType, cuuint32_t, void *,
+                                  const cuuint64_t *, const cuuint64_t *, const cuuint32_t *,
+                                  const cuuint32_t *, CUtensorMapInterleave, CUtensorMapSwizzle,
+                                  CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+inline EncodeTiledFn encode_tiled_fn() {
+  static EncodeTiledFn fn = [] {
+    void *ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) !=
+            cudaSuccess ||
+        q != cudaDriverEntryPointSuccess) {
+      cudaGetLastError();
+      return static_cast<EncodeTiledFn>(nullptr);
+    }
+    return reinterpret_cast<EncodeTiledFn>(ptr);
+  }();
+  return fn;
+}
+
+// bf16 tensor [rows][h][128] seen as a 3-D map (x = d, y = head, z = row) with
+// boxes of 64 x box_h x box_rows elements, 128-byte swizzled.
+inline bool make_map_3d(EncodeTiledFn enc, CUtensorMap *m, const void *base, uint64_t h,
+                        uint64_t rows, uint32_t box_h, uint32_t box_rows) {
+  const cuuint64_t dims[3] = {128, h, rows};
+  const cuuint64_t strides[2] = {128 * 2, h * 128 * 2};
+  const cuuint32_t box[3] = {64, box_h, box_rows};
+  const cuuint32_t es[3] = {1, 1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 3, const_cast<void *>(base), dims, strides, box,
+             es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+inline bool tc_supported(const AttnParams &p) {
+  return p.d == 128 && p.M <= 128 && p.S <= 64 && p.prefix_rows + 256 < (int64_t(1) << 31) &&
+         int64_t(p.B) * p.S + 64 < (int64_t(1) << 31);
+}
+
+inline bd_status launch_attn_tc(const AttnParams &p, cudaStream_t st) {
+  EncodeTiledFn enc = encode_tiled_fn();
+  if (!enc) return BD_ERR_CUDA;
+  const int S16 = (p.S + 15) & ~15;
+  const uint64_t blk_rows = uint64_t(p.B) * p.S;
+  // with no prefix rows at all the prefix maps are never used; point them at
+  // the block tensors so that they are still valid maps
+  const bool has_prefix = p.prefix_rows > 0;
+  const void *kp = has_prefix ? p.k_prefix : p.k_blk;
+  const void *vp = has_prefix ? p.v_prefix : p.v_blk;
+  const uint64_t prow = has_prefix ? uint64_t(p.prefix_rows) : blk_rows;
+  CUtensorMap mq, mkp, mvp, mkb, mvb;
+  if (!make_map_3d(enc, &mq, p.q, p.H_q, blk_rows, p.g, p.S) ||
+      !make_map_3d(enc, &mkp, kp, p.H_kv, prow, 1, kTcKeys) ||
+      !make_map_3d(enc, &mvp, vp, p.H_kv, prow, 1, kTcKeys) ||
+      !make_map_3d(enc, &mkb, p.k_blk, p.H_kv, blk_rows, 1, S16) ||
+      !make_map_3d(enc, &mvb, p.v_blk, p.H_kv, blk_rows, 1, S16))
+    return BD_ERR_CUDA;
+  if (cudaFuncSetAttribute(attn_tc_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           int(kTcSmemBytes)) != cudaSuccess) {
+    cudaGetLastError();
+    return BD_ERR_CUDA;
+  }
+  attn_tc_kernel<<<p.G, kTcThreads, kTcSmemBytes, st>>>(mq, mkp, mvp, mkb, mvb, p);
+  return cudaGetLastError() == cudaSuccess ? BD_OK : BD_ERR_CUDA;
+}
+
+}  // namespace bd

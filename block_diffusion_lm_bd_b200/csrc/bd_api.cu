@@ -8,6 +8,7 @@
 
 #include "attn_combine.cuh"
 #include "attn_simt.cuh"
+#include "attn_tc.cuh"
 #include "unmask.cuh"
 
 namespace {
@@ -152,7 +153,11 @@ bd_status bd_attn_step(const void *q, const void *k_prefix, const void *v_prefix
   p.max_polls = bd::kDefaultMaxPolls;
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
 
-  {
+  if (dtype == BD_DTYPE_BF16 && bd::tc_supported(p)) {
+    st = bd::launch_attn_tc(p, cs);
+    g_launches.fetch_add(1, std::memory_order_relaxed);
+    if (st != BD_OK) return st;
+  } else {
     void (*kern)(bd::AttnParams) = nullptr;
     size_t smem = 0;
     if (dtype == BD_DTYPE_F32) {
