@@ -63,6 +63,7 @@ struct AttnParams {
   AttnWs ws;
   int G;
   uint32_t max_polls;
+  int q_spread;  // tensor-core kernel: Q rows spread over the TMEM lane quadrants
 };
 
 __device__ __forceinline__ int attn_units(int L) { return (L + kUnitKeys - 1) / kUnitKeys + 1; }
@@ -75,37 +76,36 @@ struct PlanStart {
   bool bad;     // some prefix_len / prefix_offset is out of range
 };
 
-// Block-wide plan: every thread of the CTA must call it; s_scan holds
-// blockDim.x ints. The CTA's first unit is start(cta) of the partition of W.
+// Block-wide plan: every thread of the CTA must call it. s_scan: 32 ints,
+// s_misc: 4 ints of shared memory. The CTA's first unit is start(cta) of the
+// partition of W. Sequences are scanned in chunks of blockDim.x; with
+// B <= blockDim.x (the usual case) a single scan serves both passes.
 __device__ inline PlanStart attn_plan(const AttnParams &p, int cta, int *s_scan, int *s_misc) {
   const int tid = threadIdx.x;
   const int nt = blockDim.x;
-  // pass 1: total units and range check
-  int carry = 0;
-  int bad = 0;
+  if (tid == 0) {
+    s_misc[0] = 0;
+    s_misc[1] = -1;
+    s_misc[2] = 0;
+  }
+  // pass 1: total units, range check, stored scan for the combine
+  int carry = 0, bad = 0, n_mine = 0, ex_mine = 0;
   for (int base = 0; base < p.B; base += nt) {
     const int b = base + tid;
     int n = 0;
-    if (b < p.B && tid < nt) {
+    if (b < p.B) {
       const int L = p.prefix_len[b];
       const int64_t off = p.prefix_offset[b];
       if (L < 0 || off < 0 || off + L > p.prefix_rows) bad = 1;
       n = attn_units(L < 0 ? 0 : L);
     }
-    if (tid < nt) s_scan[tid] = n;
-    __syncthreads();
-    for (int o = 1; o < nt; o <<= 1) {
-      int v = (tid < nt && tid >= o) ? s_scan[tid - o] : 0;
-      __syncthreads();
-      if (tid < nt) s_scan[tid] += v;
-      __syncthreads();
-    }
-    if (cta == 0 && b < p.B && tid < nt) p.ws.cum[b] = carry + s_scan[tid] - n;
-    carry += s_scan[nt - 1];
-    __syncthreads();
+    int tot;
+    const int ex = carry + block_excl_scan(n, s_scan, &tot);
+    if (cta == 0 && b < p.B) p.ws.cum[b] = ex;
+    n_mine = n;
+    ex_mine = ex;
+    carry += tot;
   }
-  if (tid == 0) s_misc[0] = 0;
-  __syncthreads();
   if (bad) atomicOr(&s_misc[0], 1);
   __syncthreads();
   PlanStart ps;
@@ -120,37 +120,28 @@ __device__ inline PlanStart attn_plan(const AttnParams &p, int cta, int *s_scan,
   if (ps.bad || ps.W == 0) return ps;
   // pass 2: the sequence holding unit e0 = start(cta)
   const int64_t e0 = part_start(cta, ps.W, p.G);
-  if (tid == 0) {
-    s_misc[1] = -1;
-    s_misc[2] = 0;
-  }
-  carry = 0;
-  __syncthreads();
-  for (int base = 0; base < p.B; base += nt) {
-    const int b = base + tid;
-    int n = 0;
-    if (b < p.B && tid < nt) n = attn_units(max(0, p.prefix_len[b]));
-    if (tid < nt) s_scan[tid] = n;
-    __syncthreads();
-    for (int o = 1; o < nt; o <<= 1) {
-      int v = (tid < nt && tid >= o) ? s_scan[tid - o] : 0;
-      __syncthreads();
-      if (tid < nt) s_scan[tid] += v;
-      __syncthreads();
+  if (p.B <= nt) {
+    if (tid < p.B && int64_t(p.H_kv) * ex_mine <= e0 && e0 < int64_t(p.H_kv) * (ex_mine + n_mine)) {
+      s_misc[1] = tid;
+      s_misc[2] = ex_mine;
     }
-    if (b < p.B && tid < nt) {
-      const int ex = carry + s_scan[tid] - n;
-      if (int64_t(p.H_kv) * ex <= e0 && e0 < int64_t(p.H_kv) * (ex + n)) {
+  } else {
+    carry = 0;
+    for (int base = 0; base < p.B; base += nt) {
+      const int b = base + tid;
+      const int n = b < p.B ? attn_units(max(0, p.prefix_len[b])) : 0;
+      int tot;
+      const int ex = carry + block_excl_scan(n, s_scan, &tot);
+      if (b < p.B && int64_t(p.H_kv) * ex <= e0 && e0 < int64_t(p.H_kv) * (ex + n)) {
         s_misc[1] = b;
         s_misc[2] = ex;
       }
+      carry += tot;
     }
-    carry += s_scan[nt - 1];
-    __syncthreads();
   }
+  __syncthreads();
   ps.b = s_misc[1];
   ps.cum_b = s_misc[2];
-  __syncthreads();
   return ps;
 }
 

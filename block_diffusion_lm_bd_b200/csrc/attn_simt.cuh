@@ -31,7 +31,7 @@ __global__ void __launch_bounds__(kSimtThreads, 1) attn_simt_kernel(AttnParams p
   float *Ps = Vs + kSimtKeys * D;                // [kMaxRows][33]
   float *s_alpha = Ps + kMaxRows * (kSimtKeys + 1);  // [kMaxRows]
   float *s_l = s_alpha + kMaxRows;               // [kMaxRows]
-  __shared__ int s_scan[kSimtThreads];
+  __shared__ int s_scan[32];
   __shared__ int s_misc[4];
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;

@@ -16,11 +16,19 @@
 //               score tile (tcgen05.mma, A and B from shared memory), then
 //               O += P V with P read from TMEM and V from shared memory
 //               (MN-major descriptor). Also owns the TMEM allocation.
-//   warps 2-5   softmax / epilogue, one TMEM lane (= one query row) per
-//               thread: base-2 online softmax with a lazy maximum (O is
-//               rescaled only when a row maximum grows by more than 2^8),
-//               P written back over the score columns as bf16, and at the
-//               end of a segment O / l written to o (or to a boundary slot).
+//   warps 2-9   softmax / epilogue: two warps per TMEM lane quadrant (so
+//               two per SM sub-partition), each thread owning half of one
+//               query row (64 of the 128 score columns). Base-2 online softmax
+//               with a lazy maximum (O is rescaled only when a row maximum
+//               grows by more than 2^8); the two halves of a row exchange
+//               their partial maxima / sums through shared memory under a
+//               64-thread named barrier. P is written back over the score
+//               columns as bf16; at the end of a segment O / l goes to o (or
+//               to a boundary slot).
+// Row placement: TMEM lane i holds the MMA row i, and a warp can only read
+// the 32 lanes of its own sub-partition. With M = g*S <= 64 the Q rows are
+// spread 16 (= M/4) per lane quadrant by four TMA boxes, so that all four
+// sub-partitions share the softmax; with M > 64, row m sits in lane m.
 // Every mbarrier wait is bounded; a wait that runs out records
 // BD_ERR_TIMEOUT, raises a CTA-wide abort flag and the CTA drains its
 // outstanding copies / MMAs (bounded) before releasing TMEM and exiting.
@@ -31,7 +39,8 @@
 
 namespace bd {
 
-constexpr int kTcThreads = 192;
+constexpr int kTcThreads = 320;
+constexpr int kTcSoftmaxWarps = 8;
 constexpr int kTcStages = 3;
 constexpr int kTcKeys = 128;                       // keys per tile (= kUnitKeys)
 constexpr uint32_t kPanelBytes = 128 * 128;        // 128 rows x 128 B
@@ -112,8 +121,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
                    const __grid_constant__ CUtensorMap tm_vp, const __grid_constant__ CUtensorMap tm_kb,
                    const __grid_constant__ CUtensorMap tm_vb, const AttnParams p) {
   extern __shared__ uint8_t smem_raw[];
-  __shared__ int s_scan[kTcThreads];
+  __shared__ int s_scan[32];
   __shared__ int s_misc[4];
+  __shared__ float s_part[2 * 128];  // per-lane partial max / sum of the two row halves
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;
   uint8_t *smem = smem_raw + (sbase - raw);
@@ -123,16 +133,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int cta = blockIdx.x;
-  const PlanStart ps = attn_plan(p, cta, s_scan, s_misc);
-  pdl_launch_dependents();
-  if (ps.bad) {
-    if (cta == 0 && tid == 0) record_status(BD_ERR_DEVICE_ARG);
-    return;
-  }
-  if (ps.W == 0) return;
-  const int64_t e0 = part_start(cta, ps.W, p.G), e1 = part_start(cta + 1, ps.W, p.G);
-  if (e1 <= e0) return;
-
+  // set-up that does not depend on the plan first, so that it overlaps it
   if (tid == 0) {
     for (int i = 0; i < kTcStages; ++i) {
       bar_init(bars.kv_full + 8 * i, 1);
@@ -142,10 +143,10 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     bar_init(bars.q_empty, 1);
     for (int i = 0; i < 2; ++i) {
       bar_init(bars.s_full + 8 * i, 1);
-      bar_init(bars.p_full + 8 * i, 4);
+      bar_init(bars.p_full + 8 * i, kTcSoftmaxWarps);
     }
     bar_init(bars.o_ready, 1);
-    bar_init(bars.o_free, 4);
+    bar_init(bars.o_free, kTcSoftmaxWarps);
     bar_init(bars.mma_done, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -159,17 +160,24 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
+  const PlanStart ps = attn_plan(p, cta, s_scan, s_misc);  // contains __syncthreads
+  pdl_launch_dependents();
+  if (ps.bad && cta == 0 && tid == 0) record_status(BD_ERR_DEVICE_ARG);
+  const int64_t e0 = (ps.bad || ps.W == 0) ? 0 : part_start(cta, ps.W, p.G);
+  const int64_t e1 = (ps.bad || ps.W == 0) ? 0 : part_start(cta + 1, ps.W, p.G);
   tc_fence_before();
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
 
   SegWalker wk;
-  wk.init(p, ps, e0, e1);
+  if (e1 > e0) wk.init(p, ps, e0, e1);
   const uint32_t mp = p.max_polls;
   const int S16 = (p.S + 15) & ~15;
 
-  if (warp == 0) {
+  if (e1 <= e0) {
+    // no work in this CTA's range
+  } else if (warp == 0) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       uint32_t t = 0;
@@ -183,9 +191,19 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           break;
         }
         bar_expect_tx(bars.q_full, q_bytes);
-        tma_load_3d(sbase + kSmQ, &tm_q, bars.q_full, 0, wk.skv * p.g, wk.sb * p.S);
-        tma_load_3d(sbase + kSmQ + kPanelBytes, &tm_q, bars.q_full, 64, wk.skv * p.g,
-                    wk.sb * p.S);
+        if (p.q_spread) {
+          // quadrant k gets the S/4 block positions k*S/4 .. (k+1)*S/4 - 1
+          for (int k = 0; k < 4; ++k) {
+            const int z = wk.sb * p.S + k * (p.S / 4);
+            tma_load_3d(sbase + kSmQ + 32u * 128u * k, &tm_q, bars.q_full, 0, wk.skv * p.g, z);
+            tma_load_3d(sbase + kSmQ + kPanelBytes + 32u * 128u * k, &tm_q, bars.q_full, 64,
+                        wk.skv * p.g, z);
+          }
+        } else {
+          tma_load_3d(sbase + kSmQ, &tm_q, bars.q_full, 0, wk.skv * p.g, wk.sb * p.S);
+          tma_load_3d(sbase + kSmQ + kPanelBytes, &tm_q, bars.q_full, 64, wk.skv * p.g,
+                      wk.sb * p.S);
+        }
         for (int u = wk.u0; u < wk.u1; ++u, ++t) {
           const uint32_t st = t % kTcStages;
           if (t >= kTcStages &&
@@ -297,15 +315,30 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     }
   } else {
     // ------------------------------------------------------------ softmax / epilogue
-    const int q4 = warp & 3;
-    const int row = q4 * 32 + lane;
-    const bool active = q4 * 32 < p.M;  // warp-uniform
+    const int q4 = warp & 3;             // TMEM lane quadrant = SM sub-partition
+    const int hf = (warp - 2) >> 2;      // which half of the score columns
+    const int lq = q4 * 32 + lane;       // TMEM lane of this thread
+    int m;                               // packed query row of the lane
+    bool live;
+    if (p.q_spread) {
+      const int rpq = p.M >> 2;
+      live = lane < rpq;
+      m = q4 * rpq + lane;
+    } else {
+      live = lq < p.M;
+      m = lq;
+    }
+    const bool active = p.q_spread || q4 * 32 < p.M;  // same for both warps of a quadrant
     const uint32_t lrow = uint32_t(q4 * 32) << 16;
+    const uint32_t col0 = uint32_t(hf) * 64u;      // score / O columns of this half
+    const uint32_t bar_id = 1u + uint32_t(q4);     // named barrier of the quadrant's pair
+    float *x_part = s_part + (hf * 128 + lq);      // this thread's exchange slot
+    const float *x_other = s_part + ((1 - hf) * 128 + lq);
     const float c2 = p.scale_log2;
     uint32_t t = 0;
     bool ok = true;
     while (ok && wk.next(p)) {
-      float m_run = -INFINITY, l_run = 0.f;
+      float m_run = -INFINITY, l_run = 0.f;  // m_run: max of raw scores seen (unscaled)
       const int nt = wk.u1 - wk.u0;
       for (int i = 0; i < nt; ++i, ++t) {
         const int u = wk.u0 + i;
@@ -320,44 +353,50 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         float alpha = 1.f;
         bool resc = false;
         if (active) {
-          const uint32_t sc = tmem + lrow + kTmemS + 128u * sb;
-          float x[128];
+          const uint32_t sc = tmem + lrow + kTmemS + 128u * sb + col0;
+          uint32_t r[64];
+          tmem_ld_x64(sc, r);
+          float x[64];
 #pragma unroll
-          for (int c0 = 0; c0 < 128; c0 += 32) {
-            uint32_t r[32];
-            tmem_ld_x32(sc + c0, r);
+          for (int c = 0; c < 64; ++c) x[c] = __uint_as_float(r[c]);
+          const int nv = nvalid - int(col0);  // valid columns of this half (may be <= 0)
+          if (nv < 64) {
 #pragma unroll
-            for (int j = 0; j < 32; ++j) x[c0 + j] = __uint_as_float(r[j]);
+            for (int c = 0; c < 64; ++c)
+              if (c >= nv) x[c] = -INFINITY;
           }
-          float mt = -INFINITY;
+          float mx[8];
 #pragma unroll
-          for (int c = 0; c < 128; ++c) {
-            x[c] = (c < nvalid) ? x[c] * c2 : -INFINITY;
-            mt = fmaxf(mt, x[c]);
-          }
+          for (int k = 0; k < 8; ++k) mx[k] = x[k];
+#pragma unroll
+          for (int c = 8; c < 64; ++c) mx[c & 7] = fmaxf(mx[c & 7], x[c]);
+          float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                           fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+          *x_part = mt;
+          named_bar_sync(bar_id, 64);
+          mt = fmaxf(mt, *x_other);  // raw-score max of the tile row (both halves)
           if (i == 0) {
             m_run = mt;
-          } else if (mt > m_run + 8.f) {
-            alpha = exp2f(m_run - mt);
+          } else if ((mt - m_run) * c2 > 8.f) {
+            alpha = ex2_approx((m_run - mt) * c2);
             l_run *= alpha;
             m_run = mt;
             resc = true;
           }
-          float s0 = 0.f, s1 = 0.f;
+          const float nm = -m_run * c2;
+          float sm[4] = {0.f, 0.f, 0.f, 0.f};
+          uint32_t pk[32];
 #pragma unroll
-          for (int c0 = 0; c0 < 128; c0 += 64) {
-            uint32_t pk[32];
-#pragma unroll
-            for (int j = 0; j < 32; ++j) {
-              const float a = exp2f(x[c0 + 2 * j] - m_run);
-              const float b = exp2f(x[c0 + 2 * j + 1] - m_run);
-              s0 += a;
-              s1 += b;
-              pk[j] = pack_bf16x2(a, b);
-            }
-            tmem_st_x32(sc + uint32_t(c0 / 2), pk);
+          for (int j = 0; j < 32; ++j) {
+            const float a = ex2_approx(fmaf(x[2 * j], c2, nm));
+            const float b2 = ex2_approx(fmaf(x[2 * j + 1], c2, nm));
+            sm[j & 3] += a + b2;
+            pk[j] = pack_bf16x2(a, b2);
           }
-          l_run += s0 + s1;
+          l_run += (sm[0] + sm[1]) + (sm[2] + sm[3]);
+          // the partner half has loaded its scores (it passed the barrier), so
+          // P may now overwrite score columns [0, 64)
+          tmem_st_x32(tmem + lrow + kTmemS + 128u * sb + uint32_t(hf) * 32u, pk);
         }
         if (i > 0) {
           // P.V of the previous tile must be complete before O may be rescaled
@@ -368,15 +407,15 @@ __global__ void __launch_bounds__(kTcThreads, 1)
           }
           tc_fence_after();
           if (active && __any_sync(0xffffffffu, resc)) {
-            const uint32_t oc = tmem + lrow + kTmemO;
+            const uint32_t oc = tmem + lrow + kTmemO + col0;
+            uint32_t r[64];
+            tmem_ld_x64(oc, r);
 #pragma unroll
-            for (int c0 = 0; c0 < 128; c0 += 32) {
-              uint32_t r[32];
-              tmem_ld_x32(oc + c0, r);
-#pragma unroll
-              for (int j = 0; j < 32; ++j) r[j] = __float_as_uint(__uint_as_float(r[j]) * alpha);
-              tmem_st_x32(oc + c0, r);
-            }
+            for (int j = 0; j < 64; ++j) r[j] = __float_as_uint(__uint_as_float(r[j]) * alpha);
+            uint32_t (&r0)[32] = *reinterpret_cast<uint32_t (*)[32]>(&r[0]);
+            uint32_t (&r1)[32] = *reinterpret_cast<uint32_t (*)[32]>(&r[32]);
+            tmem_st_x32(oc, r0);
+            tmem_st_x32(oc + 32u, r1);
           }
         }
         tc_fence_before();
@@ -384,41 +423,40 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         if (lane == 0) bar_arrive(bars.p_full + 8 * sb);
       }
       if (!ok) break;
-      // epilogue: O / l of this segment
+      // epilogue: O / l of this segment, each half writes its 64 columns
       if (!__all_sync(0xffffffffu, tc_wait(bars.o_ready, (t - 1) & 1, mp, abort_flag))) {
         ok = false;
         break;
       }
       tc_fence_after();
       if (active) {
-        // loads are warp-wide (.sync.aligned); only rows < M store
-        const bool live = row < p.M;
-        const int m = live ? row : 0;
-        const int s = m / p.g, j = m % p.g;
-        const float inv = 1.f / l_run;
-        const float lse = (m_run + log2f(l_run)) * 0.69314718055994531f;
+        *x_part = l_run;
+        named_bar_sync(bar_id, 64);
+        const float l_tot = l_run + *x_other;
+        named_bar_sync(bar_id, 64);  // the slots are reused by the next tile's max exchange
+        const int mm = live ? m : 0;
+        const int s = mm / p.g, j = mm % p.g;
+        const float inv = 1.f / l_tot;
+        const float lse = (m_run * c2 + log2f(l_tot)) * 0.69314718055994531f;
         float *dst;
         if (wk.complete) {
-          dst = p.o + ((int64_t(wk.sb) * p.S + s) * p.H_q + wk.skv * p.g + j) * 128;
-          if (live && p.lse) p.lse[(int64_t(wk.sb) * p.H_q + wk.skv * p.g + j) * p.S + s] = lse;
+          dst = p.o + ((int64_t(wk.sb) * p.S + s) * p.H_q + wk.skv * p.g + j) * 128 + col0;
+          if (live && hf == 0 && p.lse)
+            p.lse[(int64_t(wk.sb) * p.H_q + wk.skv * p.g + j) * p.S + s] = lse;
         } else {
           const int64_t slot = attn_slot_index(cta, wk.first);
-          dst = p.ws.slot + (slot * p.M + m) * 128;
-          if (live) p.ws.slot_lse[slot * p.M + m] = lse;
+          dst = p.ws.slot + (slot * p.M + mm) * 128 + col0;
+          if (live && hf == 0) p.ws.slot_lse[slot * p.M + mm] = lse;
         }
-        const uint32_t oc = tmem + lrow + kTmemO;
+        uint32_t r[64];
+        tmem_ld_x64(tmem + lrow + kTmemO + col0, r);
+        if (live) {
 #pragma unroll
-        for (int c0 = 0; c0 < 128; c0 += 32) {
-          uint32_t r[32];
-          tmem_ld_x32(oc + c0, r);
-          if (live) {
-#pragma unroll
-            for (int j4 = 0; j4 < 8; ++j4) {
-              const float4 v = make_float4(
-                  __uint_as_float(r[4 * j4]) * inv, __uint_as_float(r[4 * j4 + 1]) * inv,
-                  __uint_as_float(r[4 * j4 + 2]) * inv, __uint_as_float(r[4 * j4 + 3]) * inv);
-              *reinterpret_cast<float4 *>(dst + c0 + 4 * j4) = v;
-            }
+          for (int j4 = 0; j4 < 16; ++j4) {
+            const float4 v = make_float4(
+                __uint_as_float(r[4 * j4]) * inv, __uint_as_float(r[4 * j4 + 1]) * inv,
+                __uint_as_float(r[4 * j4 + 2]) * inv, __uint_as_float(r[4 * j4 + 3]) * inv);
+            *reinterpret_cast<float4 *>(dst + 4 * j4) = v;
           }
         }
       }
@@ -475,7 +513,9 @@ inline bool tc_supported(const AttnParams &p) {
          int64_t(p.B) * p.S + 64 < (int64_t(1) << 31);
 }
 
-inline bd_status launch_attn_tc(const AttnParams &p, cudaStream_t st) {
+inline bd_status launch_attn_tc(AttnParams p, cudaStream_t st) {
+  // spread the rows over the four TMEM lane quadrants when they fit 16 each
+  p.q_spread = (p.M <= 64 && p.S % 4 == 0) ? 1 : 0;
   EncodeTiledFn enc = encode_tiled_fn();
   if (!enc) return BD_ERR_CUDA;
   const int S16 = (p.S + 15) & ~15;
@@ -487,7 +527,7 @@ inline bd_status launch_attn_tc(const AttnParams &p, cudaStream_t st) {
   const void *vp = has_prefix ? p.v_prefix : p.v_blk;
   const uint64_t prow = has_prefix ? uint64_t(p.prefix_rows) : blk_rows;
   CUtensorMap mq, mkp, mvp, mkb, mvb;
-  if (!make_map_3d(enc, &mq, p.q, p.H_q, blk_rows, p.g, p.S) ||
+  if (!make_map_3d(enc, &mq, p.q, p.H_q, blk_rows, p.g, p.q_spread ? p.S / 4 : p.S) ||
       !make_map_3d(enc, &mkp, kp, p.H_kv, prow, 1, kTcKeys) ||
       !make_map_3d(enc, &mvp, vp, p.H_kv, prow, 1, kTcKeys) ||
       !make_map_3d(enc, &mkb, p.k_blk, p.H_kv, blk_rows, 1, S16) ||

@@ -176,7 +176,8 @@ bd_status bd_attn_step(const void *q, const void *k_prefix, const void *v_prefix
     st = check_launch();
     if (st != BD_OK) return st;
   }
-  launch_pdl(bd::attn_combine_kernel, dim3(B * H_kv), dim3(bd::kCombineThreads), 0, cs, p);
+  launch_pdl(bd::attn_combine_kernel, dim3(B * H_kv, bd::kCombineSplit), dim3(bd::kCombineThreads), 0,
+             cs, p);
   return check_launch();
 }
 

@@ -130,6 +130,37 @@ __device__ __forceinline__ float to_f32<__nv_bfloat16>(__nv_bfloat16 x) {
   return __bfloat162float(x);
 }
 
+// Exclusive scan of one int per thread over the whole CTA (blockDim.x a
+// multiple of 32, at most 1024). s_warp: 32 ints of shared memory. Returns
+// the sum of v over the threads before this one; *total gets the CTA sum.
+// Contains three __syncthreads(); every thread must call it.
+__device__ __forceinline__ int block_excl_scan(int v, int *s_warp, int *total) {
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nwarps = blockDim.x >> 5;
+  int x = v;
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int y = __shfl_up_sync(0xffffffffu, x, o);
+    if (lane >= o) x += y;
+  }
+  if (lane == 31) s_warp[warp] = x;
+  __syncthreads();
+  if (warp == 0) {
+    int w = lane < nwarps ? s_warp[lane] : 0;
+#pragma unroll
+    for (int o = 1; o < 32; o <<= 1) {
+      const int y = __shfl_up_sync(0xffffffffu, w, o);
+      if (lane >= o) w += y;
+    }
+    s_warp[lane] = w;
+  }
+  __syncthreads();
+  const int base = warp > 0 ? s_warp[warp - 1] : 0;
+  *total = s_warp[nwarps - 1];
+  __syncthreads();
+  return base + x - v;
+}
+
 // Programmatic dependent launch: let the next kernel in the stream start its
 // prologue early / wait for the previous kernel's results.
 __device__ __forceinline__ void pdl_launch_dependents() {

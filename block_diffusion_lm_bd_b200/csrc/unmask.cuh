@@ -27,7 +27,7 @@ struct __align__(16) UnmaskPart {
   int idx;     // lowest index attaining m
 };
 
-constexpr int kUnmaskThreads = 512;
+constexpr int kUnmaskThreads = 256;
 constexpr int kUnmaskCtasPerSm = 2;
 constexpr int kUnmaskMaxRows = 65536;
 constexpr int kUnmaskRowList = 1024;  // max rows one CTA's range can touch
@@ -124,12 +124,11 @@ __device__ __forceinline__ UnmaskPart um_block_reduce(float m, int idx, double s
 
 __global__ void __launch_bounds__(kUnmaskThreads, kUnmaskCtasPerSm)
     unmask_reduce_kernel(UnmaskParams p) {
-  __shared__ int s_cnt[kUnmaskThreads];
   __shared__ int s_rows[kUnmaskRowList];
+  __shared__ int s_warp[32];
   __shared__ float sm_m[32];
   __shared__ int sm_i[32];
   __shared__ double sm_s[32];
-  __shared__ int s_total;
 
   const int tid = threadIdx.x;
   const int c = blockIdx.x;
@@ -141,18 +140,8 @@ __global__ void __launch_bounds__(kUnmaskThreads, kUnmaskCtasPerSm)
   const int r_lo = min(p.rows, tid * chunk), r_hi = min(p.rows, r_lo + chunk);
   int cnt = 0;
   for (int r = r_lo; r < r_hi; ++r) cnt += (p.mask[r] != 0);
-  s_cnt[tid] = cnt;
-  __syncthreads();
-  // Inclusive scan (Hillis-Steele) over the per-thread counts.
-  for (int o = 1; o < kUnmaskThreads; o <<= 1) {
-    int v = (tid >= o) ? s_cnt[tid - o] : 0;
-    __syncthreads();
-    s_cnt[tid] += v;
-    __syncthreads();
-  }
-  const int excl = s_cnt[tid] - cnt;
-  if (tid == kUnmaskThreads - 1) s_total = s_cnt[tid];
-  __syncthreads();
+  int s_total;
+  const int excl = block_excl_scan(cnt, s_warp, &s_total);
   const int n_masked = s_total;
   const int64_t V = p.V;
   const int64_t W = int64_t(n_masked) * V;
@@ -195,15 +184,13 @@ __global__ void __launch_bounds__(kUnmaskThreads, kUnmaskCtasPerSm)
     const int ng = (v1 - b0) >> 2;
     const float4 *x4 = reinterpret_cast<const float4 *>(x + b0);
     int g = tid;
-    for (; g + 3 * kUnmaskThreads < ng; g += 4 * kUnmaskThreads) {
-      float4 a0 = __ldcs(x4 + g);
-      float4 a1 = __ldcs(x4 + g + kUnmaskThreads);
-      float4 a2 = __ldcs(x4 + g + 2 * kUnmaskThreads);
-      float4 a3 = __ldcs(x4 + g + 3 * kUnmaskThreads);
-      um_fold4(a0, b0 + 4 * g, m, idx, s);
-      um_fold4(a1, b0 + 4 * (g + kUnmaskThreads), m, idx, s);
-      um_fold4(a2, b0 + 4 * (g + 2 * kUnmaskThreads), m, idx, s);
-      um_fold4(a3, b0 + 4 * (g + 3 * kUnmaskThreads), m, idx, s);
+    constexpr int U = 16;  // 16-byte loads in flight per thread
+    for (; g + (U - 1) * kUnmaskThreads < ng; g += U * kUnmaskThreads) {
+      float4 a[U];
+#pragma unroll
+      for (int k = 0; k < U; ++k) a[k] = __ldcs(x4 + g + k * kUnmaskThreads);
+#pragma unroll
+      for (int k = 0; k < U; ++k) um_fold4(a[k], b0 + 4 * (g + k * kUnmaskThreads), m, idx, s);
     }
     for (; g < ng; g += kUnmaskThreads) um_fold4(__ldcs(x4 + g), b0 + 4 * g, m, idx, s);
     const int t0 = b0 + 4 * ng;
