@@ -187,8 +187,9 @@ def get_device_status(stream=None, device=None):
     return int(_lib().bd_get_device_status(_stream_ptr(stream, device)))
 
 
-def debug_wait_timeout(max_polls, stream=None, device=None):
+def debug_wait_timeout(timeout_us, stream=None, device=None):
+    """Run the library's bounded-wait test kernel (see bd_debug_wait_timeout)."""
     if device is None:
         device = torch.device("cuda", torch.cuda.current_device())
-    _check(_lib().bd_debug_wait_timeout(int(max_polls), _stream_ptr(stream, device)),
+    _check(_lib().bd_debug_wait_timeout(int(timeout_us), _stream_ptr(stream, device)),
            "bd_debug_wait_timeout")

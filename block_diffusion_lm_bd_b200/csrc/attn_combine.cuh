@@ -21,6 +21,7 @@ __global__ void __launch_bounds__(kCombineThreads) attn_combine_kernel(AttnParam
   __shared__ float s_max[kMaxRows / kCombineSplit];
   __shared__ float s_den[kMaxRows / kCombineSplit];
   __shared__ int s_np;
+  pdl_launch_dependents();
   pdl_wait_previous();
   if (*p.ws.flag) return;
   const int pair = blockIdx.x;

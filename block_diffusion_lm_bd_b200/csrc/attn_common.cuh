@@ -62,7 +62,7 @@ struct AttnParams {
   float *lse;
   AttnWs ws;
   int G;
-  uint32_t max_polls;
+  uint64_t wait_ns;  // time limit of every barrier wait
   int q_spread;  // tensor-core kernel: Q rows spread over the TMEM lane quadrants
 };
 

@@ -36,6 +36,7 @@ __global__ void __launch_bounds__(kSimtThreads, 1) attn_simt_kernel(AttnParams p
 
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int cta = blockIdx.x;
+  pdl_wait_previous();
   const PlanStart ps = attn_plan(p, cta, s_scan, s_misc);
   pdl_launch_dependents();
   if (ps.bad) {

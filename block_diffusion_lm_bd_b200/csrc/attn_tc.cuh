@@ -79,25 +79,35 @@ struct TcBars {
   }
 };
 
-__device__ __forceinline__ bool tc_wait(uint32_t bar, uint32_t phase, uint32_t max_polls,
-                                        volatile int *abort_flag) {
+__device__ __forceinline__ bool tc_try(uint32_t bar, uint32_t phase) {
   uint32_t ok;
-  for (uint32_t i = 0;; ++i) {
-    asm volatile(
-        "{\n\t.reg .pred p;\n\t"
-        "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
-        "selp.u32 %0, 1, 0, p;\n\t}"
-        : "=r"(ok)
-        : "r"(bar), "r"(phase)
-        : "memory");
-    if (ok) return true;
-    if ((i & 255) == 255 && *abort_flag) return false;
-    if (i >= max_polls) {
-      record_status(BD_ERR_TIMEOUT);
-      *abort_flag = 1;
-      return false;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t}"
+      : "=r"(ok)
+      : "r"(bar), "r"(phase)
+      : "memory");
+  return ok != 0;
+}
+
+// Bounded wait on a barrier phase: gives up after limit_ns of the global timer
+// (recording BD_ERR_TIMEOUT and raising the CTA's abort flag), or as soon as
+// another role of the CTA has raised the abort flag.
+__device__ __forceinline__ bool tc_wait(uint32_t bar, uint32_t phase, uint64_t limit_ns,
+                                        volatile int *abort_flag) {
+  if (tc_try(bar, phase)) return true;
+  const uint64_t t0 = global_ns();
+  for (uint32_t i = 1;; ++i) {
+    if (tc_try(bar, phase)) return true;
+    if ((i & 255) == 0) {
+      if (*abort_flag) return false;
+      if (global_ns() - t0 > limit_ns) {
+        record_status(BD_ERR_TIMEOUT);
+        *abort_flag = 1;
+        return false;
+      }
     }
-    if (i > 256) __nanosleep(64);
   }
 }
 
@@ -160,6 +170,9 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     tmem_alloc(tmem_slot, kTmemCols);
     tmem_relinquish();
   }
+  // everything above overlaps the previous kernel of the stream; inputs are
+  // read only after it has completed
+  pdl_wait_previous();
   const PlanStart ps = attn_plan(p, cta, s_scan, s_misc);  // contains __syncthreads
   pdl_launch_dependents();
   if (ps.bad && cta == 0 && tid == 0) record_status(BD_ERR_DEVICE_ARG);
@@ -172,7 +185,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
 
   SegWalker wk;
   if (e1 > e0) wk.init(p, ps, e0, e1);
-  const uint32_t mp = p.max_polls;
+  const uint64_t mp = p.wait_ns;
   const int S16 = (p.S + 15) & ~15;
 
   if (e1 <= e0) {
@@ -538,8 +551,23 @@ inline bd_status launch_attn_tc(AttnParams p, cudaStream_t st) {
     cudaGetLastError();
     return BD_ERR_CUDA;
   }
-  attn_tc_kernel<<<p.G, kTcThreads, kTcSmemBytes, st>>>(mq, mkp, mvp, mkb, mvb, p);
-  return cudaGetLastError() == cudaSuccess ? BD_OK : BD_ERR_CUDA;
+  // programmatic dependent launch: the set-up of this kernel overlaps the tail
+  // of the previous kernel in the stream
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(p.G);
+  cfg.blockDim = dim3(kTcThreads);
+  cfg.dynamicSmemBytes = kTcSmemBytes;
+  cfg.stream = st;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, attn_tc_kernel, mq, mkp, mvp, mkb, mvb, p) != cudaSuccess) {
+    cudaGetLastError();
+    return BD_ERR_CUDA;
+  }
+  return BD_OK;
 }
 
 }  // namespace bd

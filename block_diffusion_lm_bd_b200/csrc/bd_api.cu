@@ -150,7 +150,7 @@ bd_status bd_attn_step(const void *q, const void *k_prefix, const void *v_prefix
   p.lse = lse;
   bd::attn_ws_layout(B, M, d, G, &p.ws, static_cast<char *>(workspace));
   p.G = G;
-  p.max_polls = bd::kDefaultMaxPolls;
+  p.wait_ns = bd::kDefaultWaitNs;
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
 
   if (dtype == BD_DTYPE_BF16 && bd::tc_supported(p)) {
@@ -172,7 +172,7 @@ bd_status bd_attn_step(const void *q, const void *k_prefix, const void *v_prefix
       cudaGetLastError();
       return BD_ERR_CUDA;
     }
-    kern<<<G, bd::kSimtThreads, smem, cs>>>(p);
+    launch_pdl(kern, dim3(G), dim3(bd::kSimtThreads), smem, cs, p);
     st = check_launch();
     if (st != BD_OK) return st;
   }
@@ -218,7 +218,7 @@ bd_status bd_unmask(const float *logits, const uint8_t *mask, float gamma, int32
   rp.V = V;
   rp.G = G;
   bd::unmask_ws_layout(rows, G, &rp.ws, static_cast<char *>(workspace));
-  bd::unmask_reduce_kernel<<<G, bd::kUnmaskThreads, 0, cs>>>(rp);
+  launch_pdl(bd::unmask_reduce_kernel, dim3(G), dim3(bd::kUnmaskThreads), 0, cs, rp);
   bd_status st = check_launch();
   if (st != BD_OK) return st;
 
@@ -239,7 +239,7 @@ bd_status bd_unmask(const float *logits, const uint8_t *mask, float gamma, int32
                         : bd::kUnmaskFinalizeRows;
   fp.ws = rp.ws;
   const int grid = (rows + fp.rows_per_cta - 1) / fp.rows_per_cta;
-  launch_pdl(bd::unmask_finalize_kernel, dim3(grid), dim3(bd::kUnmaskFinalizeRows), 0, cs, fp);
+  launch_pdl(bd::unmask_finalize_kernel, dim3(grid), dim3(bd::kUnmaskFinalizeThreads), 0, cs, fp);
   return check_launch();
 }
 
@@ -266,20 +266,20 @@ bd_status bd_get_device_status(bd_stream_t stream) {
 
 namespace bd {
 // The only job of this kernel: wait, bounded, on a barrier nobody arrives on.
-__global__ void debug_wait_timeout_kernel(uint32_t max_polls) {
+__global__ void debug_wait_timeout_kernel(uint64_t limit_ns) {
   __shared__ __align__(8) uint64_t bar;
   if (threadIdx.x == 0) {
     mbar_init(&bar, 1);
     fence_barrier_init();
   }
   __syncthreads();
-  if (threadIdx.x == 0) mbar_wait(&bar, 0, max_polls);
+  if (threadIdx.x == 0) mbar_wait(&bar, 0, limit_ns);
 }
 }  // namespace bd
 
-extern "C" bd_status bd_debug_wait_timeout(int max_polls, bd_stream_t stream) {
-  if (max_polls < 0) return BD_ERR_INVALID_ARG;
+extern "C" bd_status bd_debug_wait_timeout(int timeout_us, bd_stream_t stream) {
+  if (timeout_us < 0 || timeout_us > 10000000) return BD_ERR_INVALID_ARG;
   bd::debug_wait_timeout_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
-      uint32_t(max_polls));
+      uint64_t(timeout_us) * 1000ull);
   return check_launch();
 }

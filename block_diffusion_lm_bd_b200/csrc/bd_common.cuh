@@ -21,9 +21,15 @@ __device__ int g_status;
 
 __device__ __forceinline__ void record_status(int s) { atomicCAS(&g_status, 0, s); }
 
-// Default poll limit of every bounded wait (a poll costs >= ~32 ns with the
-// back-off below, so this is of the order of a second or more).
-constexpr uint32_t kDefaultMaxPolls = 1u << 25;
+// Default time limit of every bounded wait, in nanoseconds of the GPU's
+// global timer.
+constexpr uint64_t kDefaultWaitNs = 2000000000ull;
+
+__device__ __forceinline__ uint64_t global_ns() {
+  uint64_t t;
+  asm volatile("mov.u64 %0, %globaltimer;" : "=l"(t));
+  return t;
+}
 
 // ---------------------------------------------------------------------------
 // Balanced partition of W work units over G workers: worker c owns
@@ -87,12 +93,13 @@ __device__ __forceinline__ bool mbar_try_wait(uint64_t *bar, uint32_t phase) {
 }
 
 // Bounded wait for the barrier phase with parity `phase` to complete. Returns
-// false (and records BD_ERR_TIMEOUT) after max_polls unsuccessful polls.
-__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t phase, uint32_t max_polls) {
+// false (and records BD_ERR_TIMEOUT) once limit_ns have passed without it.
+__device__ __forceinline__ bool mbar_wait(uint64_t *bar, uint32_t phase, uint64_t limit_ns) {
   if (mbar_try_wait(bar, phase)) return true;
-  for (uint32_t i = 0; i < max_polls; ++i) {
+  const uint64_t t0 = global_ns();
+  for (uint32_t i = 1;; ++i) {
     if (mbar_try_wait(bar, phase)) return true;
-    if (i > 64) __nanosleep(32);
+    if ((i & 255) == 0 && global_ns() - t0 > limit_ns) break;
   }
   record_status(BD_ERR_TIMEOUT);
   return false;

@@ -31,7 +31,8 @@ constexpr int kUnmaskThreads = 256;
 constexpr int kUnmaskCtasPerSm = 2;
 constexpr int kUnmaskMaxRows = 65536;
 constexpr int kUnmaskRowList = 1024;  // max rows one CTA's range can touch
-constexpr int kUnmaskFinalizeRows = 256;
+constexpr int kUnmaskFinalizeRows = 256;   // rows per finalize CTA at most
+constexpr int kUnmaskFinalizeThreads = 256;
 
 struct UnmaskWs {
   int *n_masked;         // [1]
@@ -64,6 +65,20 @@ struct UnmaskParams {
   UnmaskWs ws;
 };
 
+// e^(x - m) as 2^((x - m) log2 e) on the special-function unit. x - m is
+// exact when x is close to m (Sterbenz), so the dominant term of a row, the
+// maximum itself, is exactly 1; the others carry a relative error of a few
+// 1e-7 at most, and terms below 2^-126 flush to zero.
+__device__ __forceinline__ float um_exp(float d) {
+  float y;
+  asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(d * 1.4426950408889634f));
+  return y;
+}
+
+__device__ __forceinline__ float um_exp_sum4(float4 x, float m) {
+  return (um_exp(x.x - m) + um_exp(x.y - m)) + (um_exp(x.z - m) + um_exp(x.w - m));
+}
+
 // Fold one value at index i into a thread's running (m, idx, s).
 __device__ __forceinline__ void um_fold1(float x, int i, float &m, int &idx, double &s) {
   if (x > m) {
@@ -71,7 +86,7 @@ __device__ __forceinline__ void um_fold1(float x, int i, float &m, int &idx, dou
     m = x;
     idx = i;
   }
-  s += double(expf(x - m));
+  s += double(um_exp(x - m));
 }
 
 // Fold four consecutive values starting at index i.
@@ -82,8 +97,20 @@ __device__ __forceinline__ void um_fold4(float4 x, int i, float &m, int &idx, do
     m = gm;
     idx = i + (x.x == gm ? 0 : (x.y == gm ? 1 : (x.z == gm ? 2 : 3)));
   }
-  float e = (expf(x.x - m) + expf(x.y - m)) + (expf(x.z - m) + expf(x.w - m));
-  s += double(e);
+  s += double(um_exp_sum4(x, m));
+}
+
+__device__ __forceinline__ void um_merge(UnmaskPart &a, const UnmaskPart &b) {
+  if (b.m > a.m) {
+    a.sum = a.sum * exp(double(a.m) - double(b.m)) + b.sum;
+    a.m = b.m;
+    a.idx = b.idx;
+  } else if (b.m < a.m) {
+    a.sum += b.sum * exp(double(b.m) - double(a.m));
+  } else {
+    a.sum += b.sum;
+    a.idx = min(a.idx, b.idx);
+  }
 }
 
 // Block-wide merge of the per-thread (m, idx, s); result valid in thread 0.
@@ -132,8 +159,10 @@ __global__ void __launch_bounds__(kUnmaskThreads, kUnmaskCtasPerSm)
 
   const int tid = threadIdx.x;
   const int c = blockIdx.x;
-  // Let the finalize kernel get launched while this grid runs.
+  // Let the finalize kernel get launched while this grid runs; wait for the
+  // previous kernel of the stream before reading anything it may have written.
   pdl_launch_dependents();
+  pdl_wait_previous();
 
   // 1. Ranks of the masked rows: each thread counts a contiguous chunk.
   const int chunk = (p.rows + kUnmaskThreads - 1) / kUnmaskThreads;
@@ -183,16 +212,48 @@ __global__ void __launch_bounds__(kUnmaskThreads, kUnmaskCtasPerSm)
     const int b0 = v0 + head;
     const int ng = (v1 - b0) >> 2;
     const float4 *x4 = reinterpret_cast<const float4 *>(x + b0);
-    int g = tid;
-    constexpr int U = 16;  // 16-byte loads in flight per thread
-    for (; g + (U - 1) * kUnmaskThreads < ng; g += U * kUnmaskThreads) {
-      float4 a[U];
+    // Batches of U 16-byte loads; the next batch is requested before the
+    // current one is folded. Per batch the maximum is folded in first (one
+    // exact fp64 rescale at most), then every value adds e^(x - m) with m fixed.
+    constexpr int U = 8;
+    float4 cur[U];
 #pragma unroll
-      for (int k = 0; k < U; ++k) a[k] = __ldcs(x4 + g + k * kUnmaskThreads);
-#pragma unroll
-      for (int k = 0; k < U; ++k) um_fold4(a[k], b0 + 4 * (g + k * kUnmaskThreads), m, idx, s);
+    for (int k = 0; k < U; ++k) {
+      const int gi = tid + k * kUnmaskThreads;
+      cur[k] = gi < ng ? __ldcs(x4 + gi) : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
     }
-    for (; g < ng; g += kUnmaskThreads) um_fold4(__ldcs(x4 + g), b0 + 4 * g, m, idx, s);
+    for (int g0 = tid; g0 < ng; g0 += U * kUnmaskThreads) {
+      float4 nxt[U];
+#pragma unroll
+      for (int k = 0; k < U; ++k) {
+        const int gi = g0 + (U + k) * kUnmaskThreads;
+        nxt[k] = gi < ng ? __ldcs(x4 + gi) : make_float4(-INFINITY, -INFINITY, -INFINITY, -INFINITY);
+      }
+      float bm = -INFINITY;
+#pragma unroll
+      for (int k = 0; k < U; ++k)
+        bm = fmaxf(bm, fmaxf(fmaxf(cur[k].x, cur[k].y), fmaxf(cur[k].z, cur[k].w)));
+      if (bm > m) {
+        s = (m == -INFINITY) ? 0.0 : s * exp(double(m) - double(bm));
+        m = bm;
+        int first = INT_MAX;  // lowest index in the batch attaining bm
+#pragma unroll
+        for (int k = U - 1; k >= 0; --k) {
+          const int e = b0 + 4 * (g0 + k * kUnmaskThreads);
+          if (cur[k].w == bm) first = e + 3;
+          if (cur[k].z == bm) first = e + 2;
+          if (cur[k].y == bm) first = e + 1;
+          if (cur[k].x == bm) first = e;
+        }
+        idx = first;
+      }
+#pragma unroll
+      for (int k = 0; k < U; ++k) {
+        if (g0 + k * kUnmaskThreads < ng) s += double(um_exp_sum4(cur[k], m));
+      }
+#pragma unroll
+      for (int k = 0; k < U; ++k) cur[k] = nxt[k];
+    }
     const int t0 = b0 + 4 * ng;
     if (t0 + tid < v1) um_fold1(__ldcs(x + t0 + tid), t0 + tid, m, idx, s);
 
@@ -222,61 +283,103 @@ struct UnmaskFinalizeParams {
   UnmaskWs ws;
 };
 
-__device__ __forceinline__ void um_merge(UnmaskPart &a, const UnmaskPart &b) {
-  if (b.m > a.m) {
-    a.sum = a.sum * exp(double(a.m) - double(b.m)) + b.sum;
-    a.m = b.m;
-    a.idx = b.idx;
-  } else if (b.m < a.m) {
-    a.sum += b.sum * exp(double(b.m) - double(a.m));
-  } else {
-    a.sum += b.sum;
-    a.idx = min(a.idx, b.idx);
-  }
+// Per row: merge the partial records, confidence, threshold. Thread t of the
+// CTA handles row t directly when the row was cut into at most kDirectParts
+// pieces (their loads are issued together); rows cut into more pieces are
+// queued and handled afterwards one warp per row, the lanes fetching the
+// records in parallel and merging them with shuffles. Then the first row of
+// every block applies the fallback, and the flags are written.
+constexpr int kDirectParts = 4;
+
+__device__ __forceinline__ void um_record_of(const UnmaskFinalizeParams &p, int64_t c, int64_t c0,
+                                             int64_t e0, int64_t W, int64_t G, UnmaskPart &a) {
+  if (c != c0 && part_start(c, W, G) == part_start(c + 1, W, G)) return;  // empty range
+  const int64_t k = (c == c0) ? 2 * c0 + (part_start(c0, W, G) == e0 ? 0 : 1) : 2 * c;
+  um_merge(a, p.ws.slot[k]);
 }
 
-__global__ void __launch_bounds__(kUnmaskFinalizeRows)
+__global__ void __launch_bounds__(kUnmaskFinalizeThreads)
     unmask_finalize_kernel(UnmaskFinalizeParams p) {
   __shared__ double s_conf[kUnmaskFinalizeRows];
   __shared__ uint8_t s_commit[kUnmaskFinalizeRows];
   __shared__ uint8_t s_mask[kUnmaskFinalizeRows];
+  __shared__ int s_queue[kUnmaskFinalizeRows];
+  __shared__ int s_nq;
+  pdl_launch_dependents();
   pdl_wait_previous();
-  const int r = blockIdx.x * p.rows_per_cta + threadIdx.x;
-  const bool in = threadIdx.x < p.rows_per_cta && r < p.rows;
-  uint8_t mk = in ? (p.mask[r] != 0) : 0;
-  uint8_t commit = 0;
-  double conf = -1.0;
-  if (mk) {
-    const int64_t V = p.V, G = p.G;
-    const int64_t W = int64_t(*p.ws.n_masked) * V;
-    const int64_t e0 = int64_t(p.ws.rank[r]) * V, e1 = e0 + V;
-    const int64_t c0 = part_owner(e0, W, G), c1 = part_owner(e1 - 1, W, G);
+  if (threadIdx.x == 0) s_nq = 0;
+  __syncthreads();
+  const int64_t V = p.V, G = p.G;
+  const int64_t W = int64_t(*p.ws.n_masked) * V;
+  for (int lr = threadIdx.x; lr < p.rows_per_cta; lr += blockDim.x) {
+    const int r = blockIdx.x * p.rows_per_cta + lr;
+    const uint8_t mk = (r < p.rows) ? (p.mask[r] != 0) : 0;
+    s_mask[lr] = mk;
+    s_commit[lr] = 0;
+    s_conf[lr] = -1.0;
+    if (!mk) continue;
+    const int64_t e0 = int64_t(p.ws.rank[r]) * V;
+    const int64_t c0 = part_owner(e0, W, G), c1 = part_owner(e0 + V - 1, W, G);
     UnmaskPart a;
     if (c0 == c1) {
       a = p.ws.row_part[r];
+    } else if (c1 - c0 < kDirectParts) {
+      a.m = -INFINITY;
+      a.sum = 0.0;
+      a.idx = INT_MAX;
+#pragma unroll
+      for (int k = 0; k < kDirectParts; ++k)
+        if (c0 + k <= c1) um_record_of(p, c0 + k, c0, e0, W, G, a);
     } else {
-      a = p.ws.slot[2 * c0 + (part_start(c0, W, G) == e0 ? 0 : 1)];
-      for (int64_t c = c0 + 1; c <= c1; ++c)
-        if (part_start(c, W, G) < part_start(c + 1, W, G)) um_merge(a, p.ws.slot[2 * c]);
+      s_queue[atomicAdd(&s_nq, 1)] = lr;
+      continue;
     }
-    conf = 1.0 / a.sum;
-    commit = conf > double(p.gamma);
+    const double conf = 1.0 / a.sum;
+    s_conf[lr] = conf;
+    s_commit[lr] = conf > double(p.gamma);
     p.tokens_out[r] = a.idx;
     p.conf_out[r] = float(conf);
   }
+  __syncthreads();
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  for (int qi = warp; qi < s_nq; qi += blockDim.x >> 5) {
+    const int lr = s_queue[qi];
+    const int r = blockIdx.x * p.rows_per_cta + lr;
+    const int64_t e0 = int64_t(p.ws.rank[r]) * V;
+    const int64_t c0 = part_owner(e0, W, G), c1 = part_owner(e0 + V - 1, W, G);
+    UnmaskPart a;
+    a.m = -INFINITY;
+    a.sum = 0.0;
+    a.idx = INT_MAX;
+    for (int64_t c = c0 + lane; c <= c1; c += 32) um_record_of(p, c, c0, e0, W, G, a);
+    float M = a.m;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    double sm = (a.m == -INFINITY) ? 0.0 : a.sum * exp(double(a.m) - double(M));
+    int ic = (a.m == M) ? a.idx : INT_MAX;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      sm += __shfl_xor_sync(0xffffffffu, sm, o);
+      ic = min(ic, __shfl_xor_sync(0xffffffffu, ic, o));
+    }
+    if (lane == 0) {
+      const double conf = 1.0 / sm;
+      s_conf[lr] = conf;
+      s_commit[lr] = conf > double(p.gamma);
+      p.tokens_out[r] = ic;
+      p.conf_out[r] = float(conf);
+    }
+  }
+  __syncthreads();
   if (p.fallback) {
-    s_conf[threadIdx.x] = conf;
-    s_commit[threadIdx.x] = commit;
-    s_mask[threadIdx.x] = mk;
-    __syncthreads();
-    // the first row of each block decides for its block
-    const int lr = threadIdx.x;
-    if (in && lr % p.block_S == 0) {
-      const int n = min(p.block_S, p.rows_per_cta - lr);
+    for (int lr = threadIdx.x * p.block_S; lr < p.rows_per_cta; lr += blockDim.x * p.block_S) {
+      const int r = blockIdx.x * p.rows_per_cta + lr;
+      if (r >= p.rows) break;
+      const int n = min(p.block_S, p.rows - r);
       bool any_masked = false, any_commit = false;
       int best = -1;
       double bc = -1.0;
-      for (int k = 0; k < n && r + k < p.rows; ++k) {
+      for (int k = 0; k < n; ++k) {
         any_masked |= s_mask[lr + k] != 0;
         any_commit |= s_commit[lr + k] != 0;
         if (s_mask[lr + k] && s_conf[lr + k] > bc) {
@@ -287,11 +390,12 @@ __global__ void __launch_bounds__(kUnmaskFinalizeRows)
       if (any_masked && !any_commit && best >= 0) s_commit[best] = 1;
     }
     __syncthreads();
-    commit = s_commit[threadIdx.x];
   }
-  if (in) {
-    p.commit_out[r] = commit;
-    if (p.mask_out) p.mask_out[r] = (mk && !commit) ? 1 : 0;
+  for (int lr = threadIdx.x; lr < p.rows_per_cta; lr += blockDim.x) {
+    const int r = blockIdx.x * p.rows_per_cta + lr;
+    if (r >= p.rows) break;
+    p.commit_out[r] = s_commit[lr];
+    if (p.mask_out) p.mask_out[r] = (s_mask[lr] && !s_commit[lr]) ? 1 : 0;
   }
 }
 

@@ -104,7 +104,7 @@ size_t bd_attn_workspace_bytes(int B, int S, int H_q, int H_kv, int d);
  *   lse          float32 [B, H_q, S]     output, or NULL
  *   workspace    >= bd_attn_workspace_bytes(B, S, H_q, H_kv, d) bytes
  * Supported: d in {64, 128}; 1 <= S <= 64; H_q % H_kv == 0;
- * (H_q/H_kv) * S <= 128; B <= 65535. Otherwise BD_ERR_UNSUPPORTED /
+ * (H_q/H_kv) * S <= 128; B <= 4096. Otherwise BD_ERR_UNSUPPORTED /
  * BD_ERR_INVALID_ARG, and nothing is launched. Offsets or lengths out of
  * range are found on the device: nothing is written and the device status
  * becomes BD_ERR_DEVICE_ARG.
@@ -150,7 +150,8 @@ size_t bd_unmask_workspace_bytes(int rows, int V);
  *   conf_out    float32 [rows]
  *   commit_out  uint8   [rows]
  *   mask_out    uint8   [rows] or NULL
- * Supported: 1 <= rows <= 65536, 1 <= V < 2^31, block_S in [0, 1024].
+ * Supported: 1 <= rows <= 65536, 1 <= V < 2^31, block_S in [0, 256]; when
+ * commit_at_least_one != 0, block_S >= 1.
  */
 bd_status bd_unmask(const float *logits, const uint8_t *mask, float gamma, int32_t *tokens_out,
                     float *conf_out, uint8_t *commit_out, uint8_t *mask_out, int rows, int V,
@@ -178,11 +179,12 @@ uint64_t bd_launch_count(void);
 /*
  * Test hook for the failure path: launches one tiny kernel whose only job is
  * a bounded wait on a shared-memory barrier that nothing ever arrives on.
- * The wait gives up after `max_polls` polls, records BD_ERR_TIMEOUT in the
- * device status word and returns, leaving the context usable. Read the
- * result with bd_get_device_status.
+ * The wait gives up after `timeout_us` microseconds (0 .. 10^7), records
+ * BD_ERR_TIMEOUT in the device status word and returns, leaving the context
+ * usable. Read the result with bd_get_device_status. Every wait inside the
+ * library's kernels is bounded the same way (2 s).
  */
-bd_status bd_debug_wait_timeout(int max_polls, bd_stream_t stream);
+bd_status bd_debug_wait_timeout(int timeout_us, bd_stream_t stream);
 
 #ifdef __cplusplus
 }

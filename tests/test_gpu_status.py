@@ -15,7 +15,7 @@ pytestmark = pytest.mark.gpu
 
 def test_bounded_wait_times_out_and_context_survives():
     assert api.get_device_status() == 0
-    api.debug_wait_timeout(1000)
+    api.debug_wait_timeout(2000)  # 2 ms
     assert api.get_device_status() == 4  # BD_ERR_TIMEOUT
     assert api.get_device_status() == 0  # cleared
     x = torch.randn(4, 1000, device="cuda")
