@@ -33,7 +33,7 @@ struct AttnWs {
 
 __host__ __device__ inline size_t attn_align(size_t x) { return (x + 255) & ~size_t(255); }
 
-__host__ __device__ inline size_t attn_ws_layout(int B, int M, int d, int G, AttnWs *ws,
+__host__ __device__ inline size_t attn_ws_layout(int B, int H_kv, int M, int d, int G, AttnWs *ws,
                                                  char *base) {
   size_t off = 0;
   if (ws) ws->flag = reinterpret_cast<int *>(base + off);
@@ -153,7 +153,7 @@ struct SegWalker {
   int64_t off;
   // the segment returned by the last next()
   int sb, skv, sL, sn, u0, u1;
-  int64_t soff;
+  int64_t soff, spbase;
   bool first, complete;
 
   __device__ void init(const AttnParams &p, const PlanStart &ps, int64_t e0_, int64_t e1_) {
@@ -180,6 +180,7 @@ struct SegWalker {
     sL = L;
     sn = n;
     soff = off;
+    spbase = pbase;
     e = pbase + u1;
     if (++kv == p.H_kv) {
       kv = 0;
@@ -192,6 +193,33 @@ struct SegWalker {
       }
     }
     return true;
+  }
+};
+
+// The CTAs c0 .. c1 that hold parts of the pair whose units are
+// [base, base + n), and the boundary slot of each part. When every CTA range
+// is non-empty (W >= G) the slot of CTA c > c0 is simply 2c (its first
+// segment); only c0 needs a test. With W < G, CTAs with empty ranges are
+// skipped (slot -1).
+struct PairParts {
+  int64_t c0, c1, s0;
+  bool dense;
+  __device__ PairParts(int64_t base, int n, int64_t W, int64_t G) {
+    c0 = part_owner(base, W, G);
+    c1 = part_owner(base + n - 1, W, G);
+    s0 = 2 * c0 + (part_start(c0, W, G) == base ? 0 : 1);
+    dense = W >= G;
+  }
+  __device__ int64_t slot(int64_t c, int64_t W, int64_t G) const {
+    if (c == c0) return s0;
+    if (dense || part_start(c, W, G) < part_start(c + 1, W, G)) return 2 * c;
+    return -1;
+  }
+  __device__ int count(int64_t W, int64_t G) const {
+    if (dense) return int(c1 - c0 + 1);
+    int np = 1;
+    for (int64_t c = c0 + 1; c <= c1; ++c) np += part_start(c, W, G) < part_start(c + 1, W, G);
+    return np;
   }
 };
 

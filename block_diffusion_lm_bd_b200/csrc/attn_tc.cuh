@@ -349,17 +349,18 @@ __global__ void __launch_bounds__(kTcThreads, 1)
     const float *x_other = s_part + ((1 - hf) * 128 + lq);
     const float c2 = p.scale_log2;
     uint32_t t = 0;
+    // Once a wait fails (timeout or abort) the warp is poisoned: it skips every
+    // wait, TMEM access and store, but still walks the same segments and
+    // executes the same named barriers, so that no partner warp can be left
+    // waiting in a bar.sync.
     bool ok = true;
-    while (ok && wk.next(p)) {
+    while (wk.next(p)) {
       float m_run = -INFINITY, l_run = 0.f;  // m_run: max of raw scores seen (unscaled)
       const int nt = wk.u1 - wk.u0;
       for (int i = 0; i < nt; ++i, ++t) {
         const int u = wk.u0 + i;
         const uint32_t sb = t & 1;
-        if (!__all_sync(0xffffffffu, tc_wait(bars.s_full + 8 * sb, (t >> 1) & 1, mp, abort_flag))) {
-          ok = false;
-          break;
-        }
+        ok = ok && __all_sync(0xffffffffu, tc_wait(bars.s_full + 8 * sb, (t >> 1) & 1, mp, abort_flag));
         tc_fence_after();
         const bool blk = (u == wk.sn - 1);
         const int nvalid = blk ? p.S : min(kTcKeys, wk.sL - u * kTcKeys);
@@ -367,59 +368,61 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         bool resc = false;
         if (active) {
           const uint32_t sc = tmem + lrow + kTmemS + 128u * sb + col0;
-          uint32_t r[64];
-          tmem_ld_x64(sc, r);
           float x[64];
+          float mt = -INFINITY;
+          if (ok) {
+            uint32_t r[64];
+            tmem_ld_x64(sc, r);
 #pragma unroll
-          for (int c = 0; c < 64; ++c) x[c] = __uint_as_float(r[c]);
-          const int nv = nvalid - int(col0);  // valid columns of this half (may be <= 0)
-          if (nv < 64) {
+            for (int c = 0; c < 64; ++c) x[c] = __uint_as_float(r[c]);
+            const int nv = nvalid - int(col0);  // valid columns of this half (may be <= 0)
+            if (nv < 64) {
 #pragma unroll
-            for (int c = 0; c < 64; ++c)
-              if (c >= nv) x[c] = -INFINITY;
+              for (int c = 0; c < 64; ++c)
+                if (c >= nv) x[c] = -INFINITY;
+            }
+            float mx[8];
+#pragma unroll
+            for (int k = 0; k < 8; ++k) mx[k] = x[k];
+#pragma unroll
+            for (int c = 8; c < 64; ++c) mx[c & 7] = fmaxf(mx[c & 7], x[c]);
+            mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                       fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
           }
-          float mx[8];
-#pragma unroll
-          for (int k = 0; k < 8; ++k) mx[k] = x[k];
-#pragma unroll
-          for (int c = 8; c < 64; ++c) mx[c & 7] = fmaxf(mx[c & 7], x[c]);
-          float mt = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
-                           fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
           *x_part = mt;
           named_bar_sync(bar_id, 64);
           mt = fmaxf(mt, *x_other);  // raw-score max of the tile row (both halves)
-          if (i == 0) {
-            m_run = mt;
-          } else if ((mt - m_run) * c2 > 8.f) {
-            alpha = ex2_approx((m_run - mt) * c2);
-            l_run *= alpha;
-            m_run = mt;
-            resc = true;
-          }
-          const float nm = -m_run * c2;
-          float sm[4] = {0.f, 0.f, 0.f, 0.f};
-          uint32_t pk[32];
+          if (ok) {
+            if (i == 0) {
+              m_run = mt;
+            } else if ((mt - m_run) * c2 > 8.f) {
+              alpha = ex2_approx((m_run - mt) * c2);
+              l_run *= alpha;
+              m_run = mt;
+              resc = true;
+            }
+            const float nm = -m_run * c2;
+            float sm[4] = {0.f, 0.f, 0.f, 0.f};
+            uint32_t pk[32];
 #pragma unroll
-          for (int j = 0; j < 32; ++j) {
-            const float a = ex2_approx(fmaf(x[2 * j], c2, nm));
-            const float b2 = ex2_approx(fmaf(x[2 * j + 1], c2, nm));
-            sm[j & 3] += a + b2;
-            pk[j] = pack_bf16x2(a, b2);
+            for (int j = 0; j < 32; ++j) {
+              const float a = ex2_approx(fmaf(x[2 * j], c2, nm));
+              const float b2 = ex2_approx(fmaf(x[2 * j + 1], c2, nm));
+              sm[j & 3] += a + b2;
+              pk[j] = pack_bf16x2(a, b2);
+            }
+            l_run += (sm[0] + sm[1]) + (sm[2] + sm[3]);
+            // the partner half has loaded its scores (it passed the barrier), so
+            // P may now overwrite score columns [0, 64)
+            tmem_st_x32(tmem + lrow + kTmemS + 128u * sb + uint32_t(hf) * 32u, pk);
           }
-          l_run += (sm[0] + sm[1]) + (sm[2] + sm[3]);
-          // the partner half has loaded its scores (it passed the barrier), so
-          // P may now overwrite score columns [0, 64)
-          tmem_st_x32(tmem + lrow + kTmemS + 128u * sb + uint32_t(hf) * 32u, pk);
         }
         if (i > 0) {
           // P.V of the previous tile must be complete before O may be rescaled
           // and before the next P.V is released
-          if (!__all_sync(0xffffffffu, tc_wait(bars.o_ready, (t - 1) & 1, mp, abort_flag))) {
-            ok = false;
-            break;
-          }
+          ok = ok && __all_sync(0xffffffffu, tc_wait(bars.o_ready, (t - 1) & 1, mp, abort_flag));
           tc_fence_after();
-          if (active && __any_sync(0xffffffffu, resc)) {
+          if (ok && active && __any_sync(0xffffffffu, resc)) {
             const uint32_t oc = tmem + lrow + kTmemO + col0;
             uint32_t r[64];
             tmem_ld_x64(oc, r);
@@ -435,41 +438,39 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         __syncwarp();
         if (lane == 0) bar_arrive(bars.p_full + 8 * sb);
       }
-      if (!ok) break;
       // epilogue: O / l of this segment, each half writes its 64 columns
-      if (!__all_sync(0xffffffffu, tc_wait(bars.o_ready, (t - 1) & 1, mp, abort_flag))) {
-        ok = false;
-        break;
-      }
+      ok = ok && __all_sync(0xffffffffu, tc_wait(bars.o_ready, (t - 1) & 1, mp, abort_flag));
       tc_fence_after();
       if (active) {
         *x_part = l_run;
         named_bar_sync(bar_id, 64);
         const float l_tot = l_run + *x_other;
         named_bar_sync(bar_id, 64);  // the slots are reused by the next tile's max exchange
-        const int mm = live ? m : 0;
-        const int s = mm / p.g, j = mm % p.g;
-        const float inv = 1.f / l_tot;
-        const float lse = (m_run * c2 + log2f(l_tot)) * 0.69314718055994531f;
-        float *dst;
-        if (wk.complete) {
-          dst = p.o + ((int64_t(wk.sb) * p.S + s) * p.H_q + wk.skv * p.g + j) * 128 + col0;
-          if (live && hf == 0 && p.lse)
-            p.lse[(int64_t(wk.sb) * p.H_q + wk.skv * p.g + j) * p.S + s] = lse;
-        } else {
-          const int64_t slot = attn_slot_index(cta, wk.first);
-          dst = p.ws.slot + (slot * p.M + mm) * 128 + col0;
-          if (live && hf == 0) p.ws.slot_lse[slot * p.M + mm] = lse;
-        }
-        uint32_t r[64];
-        tmem_ld_x64(tmem + lrow + kTmemO + col0, r);
-        if (live) {
+        if (ok) {
+          const int mm = live ? m : 0;
+          const int s = mm / p.g, j = mm % p.g;
+          const float inv = 1.f / l_tot;
+          const float lse = (m_run * c2 + log2f(l_tot)) * 0.69314718055994531f;
+          float *dst;
+          if (wk.complete) {
+            dst = p.o + ((int64_t(wk.sb) * p.S + s) * p.H_q + wk.skv * p.g + j) * 128 + col0;
+            if (live && hf == 0 && p.lse)
+              p.lse[(int64_t(wk.sb) * p.H_q + wk.skv * p.g + j) * p.S + s] = lse;
+          } else {
+            const int64_t slot = attn_slot_index(cta, wk.first);
+            dst = p.ws.slot + (slot * p.M + mm) * 128 + col0;
+            if (live && hf == 0) p.ws.slot_lse[slot * p.M + mm] = lse;
+          }
+          uint32_t r[64];
+          tmem_ld_x64(tmem + lrow + kTmemO + col0, r);
+          if (live) {
 #pragma unroll
-          for (int j4 = 0; j4 < 16; ++j4) {
-            const float4 v = make_float4(
-                __uint_as_float(r[4 * j4]) * inv, __uint_as_float(r[4 * j4 + 1]) * inv,
-                __uint_as_float(r[4 * j4 + 2]) * inv, __uint_as_float(r[4 * j4 + 3]) * inv);
-            *reinterpret_cast<float4 *>(dst + 4 * j4) = v;
+            for (int j4 = 0; j4 < 16; ++j4) {
+              const float4 v = make_float4(
+                  __uint_as_float(r[4 * j4]) * inv, __uint_as_float(r[4 * j4 + 1]) * inv,
+                  __uint_as_float(r[4 * j4 + 2]) * inv, __uint_as_float(r[4 * j4 + 3]) * inv);
+              *reinterpret_cast<float4 *>(dst + 4 * j4) = v;
+            }
           }
         }
       }
@@ -522,7 +523,7 @@ inline bool make_map_3d(EncodeTiledFn enc, CUtensorMap *m, const void *base, uin
 }
 
 inline bool tc_supported(const AttnParams &p) {
-  return p.d == 128 && p.M <= 128 && p.S <= 64 && p.prefix_rows + 256 < (int64_t(1) << 31) &&
+  return p.G <= 255 && p.d == 128 && p.M <= 128 && p.S <= 64 && p.prefix_rows + 256 < (int64_t(1) << 31) &&
          int64_t(p.B) * p.S + 64 < (int64_t(1) << 31);
 }
 
@@ -551,22 +552,10 @@ inline bd_status launch_attn_tc(AttnParams p, cudaStream_t st) {
     cudaGetLastError();
     return BD_ERR_CUDA;
   }
-  // programmatic dependent launch: the set-up of this kernel overlaps the tail
-  // of the previous kernel in the stream
-  cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(p.G);
-  cfg.blockDim = dim3(kTcThreads);
-  cfg.dynamicSmemBytes = kTcSmemBytes;
-  cfg.stream = st;
-  cudaLaunchAttribute attr[1];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, attn_tc_kernel, mq, mkp, mvp, mkb, mvb, p) != cudaSuccess) {
-    cudaGetLastError();
-    return BD_ERR_CUDA;
-  }
+  // A plain launch: measured on B200, letting this kernel (one 227 KB CTA per
+  // SM) start early under programmatic stream serialisation made steps slower.
+  attn_tc_kernel<<<p.G, kTcThreads, kTcSmemBytes, st>>>(mq, mkp, mvp, mkb, mvb, p);
+  if (cudaGetLastError() != cudaSuccess) return BD_ERR_CUDA;
   return BD_OK;
 }
 

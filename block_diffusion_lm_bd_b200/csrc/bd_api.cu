@@ -15,6 +15,7 @@ namespace {
 
 std::atomic<uint64_t> g_launches{0};
 
+
 inline bool aligned16(const void *p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
 // SM count of the current device, or 0 when no device is usable.
@@ -97,7 +98,7 @@ size_t bd_attn_workspace_bytes(int B, int S, int H_q, int H_kv, int d) {
   const int sms = sm_count();
   if (sms <= 0) return 0;
   const int M = (H_q / H_kv) * S;
-  return bd::attn_ws_layout(B, M, d, attn_grid(sms), nullptr, nullptr);
+  return bd::attn_ws_layout(B, H_kv, M, d, attn_grid(sms), nullptr, nullptr);
 }
 
 bd_status bd_attn_step(const void *q, const void *k_prefix, const void *v_prefix,
@@ -125,7 +126,7 @@ bd_status bd_attn_step(const void *q, const void *k_prefix, const void *v_prefix
   if (sms <= 0) return BD_ERR_CUDA;
   const int G = attn_grid(sms);
   const int g = H_q / H_kv, M = g * S;
-  if (workspace_bytes < bd::attn_ws_layout(B, M, d, G, nullptr, nullptr))
+  if (workspace_bytes < bd::attn_ws_layout(B, H_kv, M, d, G, nullptr, nullptr))
     return BD_ERR_INVALID_ARG;
 
   bd::AttnParams p = {};
@@ -148,7 +149,7 @@ bd_status bd_attn_step(const void *q, const void *k_prefix, const void *v_prefix
   p.scale_log2 = sc * 1.4426950408889634f;
   p.o = o;
   p.lse = lse;
-  bd::attn_ws_layout(B, M, d, G, &p.ws, static_cast<char *>(workspace));
+  bd::attn_ws_layout(B, H_kv, M, d, G, &p.ws, static_cast<char *>(workspace));
   p.G = G;
   p.wait_ns = bd::kDefaultWaitNs;
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
@@ -172,12 +173,12 @@ bd_status bd_attn_step(const void *q, const void *k_prefix, const void *v_prefix
       cudaGetLastError();
       return BD_ERR_CUDA;
     }
-    launch_pdl(kern, dim3(G), dim3(bd::kSimtThreads), smem, cs, p);
+    kern<<<G, bd::kSimtThreads, smem, cs>>>(p);
     st = check_launch();
     if (st != BD_OK) return st;
   }
-  launch_pdl(bd::attn_combine_kernel, dim3(B * H_kv, bd::kCombineSplit), dim3(bd::kCombineThreads), 0,
-             cs, p);
+  bd::attn_combine_kernel<<<dim3(B * H_kv, (M + bd::kCombineRows - 1) / bd::kCombineRows),
+                            bd::kCombineThreads, 0, cs>>>(p);
   return check_launch();
 }
 
