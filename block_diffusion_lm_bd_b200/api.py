@@ -53,6 +53,8 @@ def _lib():
     lib.bd_unmask_workspace_bytes.argtypes = [i32, i32]
     lib.bd_unmask.restype = i32
     lib.bd_unmask.argtypes = [vp, vp, f32, vp, vp, vp, vp, i32, i32, i32, i32, vp, sz, vp]
+    lib.bd_unmask_noalloc.restype = i32
+    lib.bd_unmask_noalloc.argtypes = [vp, vp, f32, vp, vp, vp, vp, i32, i32, i32, i32, vp]
     lib.bd_get_device_status.restype = i32
     lib.bd_get_device_status.argtypes = [vp]
     lib.bd_debug_wait_timeout.restype = i32
@@ -177,6 +179,32 @@ def unmask(logits, mask, gamma, block_S=0, commit_at_least_one=False, tokens_out
         _ptr(commit_out), _ptr(mask_out), rows, V, int(block_S), 1 if commit_at_least_one else 0,
         _ptr(workspace), workspace.numel() * workspace.element_size(), _stream_ptr(stream, dev))
     _check(st, "bd_unmask")
+    return {"tokens": tokens_out, "conf": conf_out, "commit": commit_out, "mask_out": mask_out}
+
+
+def unmask_noalloc(logits, mask, gamma, block_S=0, commit_at_least_one=False, tokens_out=None,
+                   conf_out=None, commit_out=None, mask_out=None, stream=None):
+    """bd_unmask_noalloc on torch tensors: like unmask(), with the library's
+    fixed scratch instead of a workspace (for callers that cannot allocate
+    device memory while they unmask). At most 16384 rows; calls that overlap
+    on the GPU must not happen (they share the scratch)."""
+    rows, V = logits.shape
+    dev = logits.device
+    _need(logits, "logits", torch.float32)
+    _need(mask, "mask", torch.uint8, dev)
+    if tokens_out is None:
+        tokens_out = torch.full((rows,), -1, dtype=torch.int32, device=dev)
+    if conf_out is None:
+        conf_out = torch.full((rows,), float("nan"), dtype=torch.float32, device=dev)
+    if commit_out is None:
+        commit_out = torch.empty((rows,), dtype=torch.uint8, device=dev)
+    if isinstance(mask_out, str) and mask_out == "inplace":
+        mask_out = mask
+    st = _lib().bd_unmask_noalloc(
+        _ptr(logits), _ptr(mask), float(gamma), _ptr(tokens_out), _ptr(conf_out),
+        _ptr(commit_out), _ptr(mask_out), rows, V, int(block_S), 1 if commit_at_least_one else 0,
+        _stream_ptr(stream, dev))
+    _check(st, "bd_unmask_noalloc")
     return {"tokens": tokens_out, "conf": conf_out, "commit": commit_out, "mask_out": mask_out}
 
 

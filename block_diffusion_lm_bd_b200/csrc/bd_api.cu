@@ -5,6 +5,7 @@
 #include <atomic>
 #include <cmath>
 #include <cstdio>
+#include <mutex>
 
 #include "attn_combine.cuh"
 #include "attn_simt.cuh"
@@ -283,4 +284,79 @@ extern "C" bd_status bd_debug_wait_timeout(int timeout_us, bd_stream_t stream) {
   bd::debug_wait_timeout_kernel<<<1, 32, 0, reinterpret_cast<cudaStream_t>(stream)>>>(
       uint64_t(timeout_us) * 1000ull);
   return check_launch();
+}
+
+// ---------------------------------------------------------------------------
+// Allocation-free unmasking.
+//
+// Some callers cannot allocate device memory at the moment they unmask: code
+// running inside another runtime's execution hook (an inference server's
+// custom operator or a plugin) that must keep its memory footprint fixed and
+// may not call the allocator while it runs, or a host program whose language
+// binding has no CUDA allocator at all. For them bd_unmask_noalloc takes its
+// scratch from a fixed array compiled into this library instead of from a
+// caller-provided workspace.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kNoAllocScratchBytes = 512 * 1024;  // held on every device that loads the library
+constexpr int kNoAllocMaxRows = 16384;
+constexpr int kNoAllocMaxDevices = 64;
+
+// In host code this name is only a stand-in: its device address comes from
+// cudaGetSymbolAddress below.
+static __device__ __align__(256) unsigned char g_unmask_scratch[kNoAllocScratchBytes];
+
+std::mutex g_scratch_mutex;
+void *g_scratch_addr[kNoAllocMaxDevices];  // device address per device, once set up
+
+// Set-up, once per device, with that device current.
+bd_status unmask_scratch_address(void **out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return BD_ERR_CUDA;
+  }
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return BD_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lock(g_scratch_mutex);
+  if (g_scratch_addr[dev] == nullptr) {
+    void *ptr = nullptr;
+    const cudaError_t e = cudaGetSymbolAddress(&ptr, g_unmask_scratch);
+    if (e != cudaSuccess || ptr == nullptr) {
+      cudaGetLastError();
+      std::fprintf(stderr, "libbd: cudaGetSymbolAddress of the unmask scratch failed: %s\n",
+                   cudaGetErrorString(e));
+      return BD_ERR_CUDA;
+    }
+    g_scratch_addr[dev] = ptr;
+  }
+  *out = g_scratch_addr[dev];
+  return BD_OK;
+}
+
+}  // namespace
+
+extern "C" bd_status bd_unmask_noalloc(const float *logits, const uint8_t *mask, float gamma,
+                                       int32_t *tokens_out, float *conf_out, uint8_t *commit_out,
+                                       uint8_t *mask_out, int rows, int V, int block_S,
+                                       int commit_at_least_one, bd_stream_t stream) {
+  if (rows > kNoAllocMaxRows) {
+    std::fprintf(stderr, "libbd: bd_unmask_noalloc supports at most %d rows (got %d)\n",
+                 kNoAllocMaxRows, rows);
+    return BD_ERR_UNSUPPORTED;
+  }
+  if (rows < 0 || V < 1) return BD_ERR_INVALID_ARG;
+  if (rows == 0) return BD_OK;
+  const int sms = sm_count();
+  if (sms <= 0) return BD_ERR_CUDA;
+  if (bd::unmask_ws_layout(rows, unmask_grid(sms), nullptr, nullptr) > kNoAllocScratchBytes) {
+    std::fprintf(stderr, "libbd: bd_unmask_noalloc scratch of %zu bytes is too small here\n",
+                 kNoAllocScratchBytes);
+    return BD_ERR_UNSUPPORTED;
+  }
+  void *scratch = nullptr;
+  const bd_status st = unmask_scratch_address(&scratch);
+  if (st != BD_OK) return st;
+  return bd_unmask(logits, mask, gamma, tokens_out, conf_out, commit_out, mask_out, rows, V,
+                   block_S, commit_at_least_one, scratch, kNoAllocScratchBytes, stream);
 }

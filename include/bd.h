@@ -158,6 +158,31 @@ bd_status bd_unmask(const float *logits, const uint8_t *mask, float gamma, int32
                     int block_S, int commit_at_least_one, void *workspace,
                     size_t workspace_bytes, bd_stream_t stream);
 
+/*
+ * bd_unmask without a workspace argument, for callers that cannot allocate
+ * device memory when they unmask: code running inside another runtime's
+ * execution hook (a server's custom operator, a plugin) that must keep its
+ * memory footprint fixed and may not call the allocator there, or a host
+ * program whose language binding has no CUDA allocator. (The source pages
+ * have no counterpart of this entry point; it is a deployment convenience.)
+ *
+ * Same arguments, results and errors as bd_unmask, minus the workspace: the
+ * scratch is a fixed 512 KiB array compiled into the library, which every GPU
+ * that loads the library holds until the process exits. It allocates nothing
+ * and frees nothing.
+ *   - rows <= 16384; more returns BD_ERR_UNSUPPORTED (and prints why).
+ *   - The first call on each device looks the array's device address up
+ *     (cudaGetSymbolAddress, with that device current) and keeps it; make that
+ *     first call before any stream capture.
+ *   - Every call, on every stream, shares the one array, which keeps the last
+ *     call's contents (nothing in it needs to start at zero). Calls that
+ *     overlap on the GPU race on it: serialise them (one stream, or events).
+ */
+bd_status bd_unmask_noalloc(const float *logits, const uint8_t *mask, float gamma,
+                            int32_t *tokens_out, float *conf_out, uint8_t *commit_out,
+                            uint8_t *mask_out, int rows, int V, int block_S,
+                            int commit_at_least_one, bd_stream_t stream);
+
 /* ------------------------------------------------------------------------ */
 /* Status, diagnostics                                                      */
 /* ------------------------------------------------------------------------ */

@@ -1,0 +1,74 @@
+"""bd_unmask_noalloc: unmasking for callers that cannot allocate device memory
+while they run (an execution hook of another runtime that must keep a fixed
+memory footprint, or a host language without a CUDA allocator).
+
+The entry point is called through the C ABI (ctypes) twice in a row, with
+different inputs, and each time its outputs must equal those of bd_unmask
+(the workspace entry point) within the unmask tolerances of the other tests:
+token ids and commit flags identical, confidences within 1e-6. This file is
+collected last so that a run that stops at the first failure has already run
+every other test; it also passes alone in a fresh process (the first call on
+the device performs the scratch set-up).
+"""
+
+import ctypes
+
+import numpy as np
+import pytest
+import torch
+
+from block_diffusion_lm_bd_b200 import api, workloads
+from _util import CONF_TOL
+
+pytestmark = pytest.mark.gpu
+DEV = torch.device("cuda", 0)
+
+
+def _call_noalloc(logits, mask, gamma, block_S, fallback, stream):
+    lib = api._lib()
+    rows, V = logits.shape
+    tok = torch.full((rows,), -7, dtype=torch.int32, device=DEV)
+    conf = torch.full((rows,), -7.0, dtype=torch.float32, device=DEV)
+    com = torch.full((rows,), 9, dtype=torch.uint8, device=DEV)
+    mo = torch.full((rows,), 9, dtype=torch.uint8, device=DEV)
+    p = lambda t: ctypes.c_void_p(t.data_ptr())
+    st = lib.bd_unmask_noalloc(p(logits), p(mask), ctypes.c_float(gamma), p(tok), p(conf), p(com),
+                               p(mo), rows, V, block_S, 1 if fallback else 0,
+                               ctypes.c_void_p(stream.cuda_stream))
+    assert st == 0, api.status_string(st)
+    return tok, conf, com, mo
+
+
+@pytest.mark.parametrize("fallback", [False, True])
+def test_noalloc_equals_workspace_entry_point_on_two_calls(fallback):
+    stream = torch.cuda.current_stream(DEV)
+    w = workloads.WORKLOADS[4 if fallback else 1]
+    for call in range(2):
+        rows = 1024 if fallback else 128
+        logits = workloads.logits(w, device=DEV, step=call, rows=rows)
+        g = torch.Generator().manual_seed(call)
+        mask = (torch.rand(rows, generator=g) < 0.8).to(torch.uint8).to(DEV)
+        tok, conf, com, mo = _call_noalloc(logits, mask, w.gamma, w.S, fallback, stream)
+        ref = api.unmask(logits, mask, w.gamma, block_S=w.S, commit_at_least_one=fallback,
+                         mask_out=torch.empty_like(mask))
+        torch.cuda.synchronize()
+        assert api.get_device_status() == 0
+        m = mask.cpu().numpy().astype(bool)
+        assert (tok.cpu().numpy()[m] == ref["tokens"].cpu().numpy()[m]).all()
+        assert (tok.cpu().numpy()[~m] == -7).all(), "unmasked rows must be left untouched"
+        cg, cr = conf.cpu().numpy()[m].astype(np.float64), ref["conf"].cpu().numpy()[m]
+        assert np.abs(cg - cr).max() <= CONF_TOL
+        assert (com.cpu().numpy() == ref["commit"].cpu().numpy()).all()
+        assert (mo.cpu().numpy() == ref["mask_out"].cpu().numpy()).all()
+
+
+def test_noalloc_rejects_more_rows_than_its_scratch_holds():
+    lib = api._lib()
+    rows, V = 16385, 8
+    logits = torch.zeros(rows, V, device=DEV)
+    mask = torch.ones(rows, dtype=torch.uint8, device=DEV)
+    out = torch.empty(rows, dtype=torch.int32, device=DEV)
+    p = lambda t: ctypes.c_void_p(t.data_ptr())
+    st = lib.bd_unmask_noalloc(p(logits), p(mask), ctypes.c_float(0.5), p(out), p(out), p(mask),
+                               None, rows, V, 0, 0, None)
+    assert st == 2  # BD_ERR_UNSUPPORTED
