@@ -92,6 +92,15 @@ def max_over_ranks(x, dist, device=None):
     return float(t.item())
 
 
+def aggregate_throughput(units_per_rank, ms_local, dist, device=None):
+    """Whole-job throughput of independent replicas: the units all ranks
+    processed divided by the slowest rank's device time. Returns (units/s,
+    max ms)."""
+    world = 1 if dist is None else dist.get_world_size()
+    ms = max_over_ranks(ms_local, dist, device)
+    return units_per_rank * world / (ms * 1e-3), ms
+
+
 def barrier(dist, device=None):
     if dist is not None:
         if device is not None and device.type == "cuda":
@@ -206,7 +215,7 @@ def run_gpu(args):
         _build.build()
     barrier(dist, dev)
     w = workloads.WORKLOADS[args.workload]
-    nsets = 4
+    nsets = args.sets
     sets = make_sets(w, dev, nsets, rank)
     lens = sets[0]["prefix_len_host"].tolist()
     B, S, H_q, H_kv, d, V = w.B, w.S, w.H_q, w.H_kv, w.d, w.V
@@ -286,7 +295,7 @@ def run_gpu(args):
     if st != 0:
         raise RuntimeError(f"device status {api.status_string(st)}")
     ms_local = t0.elapsed_time(t1)
-    ms = max_over_ranks(ms_local, dist, dev)
+    value, ms = aggregate_throughput(rows * args.steps, ms_local, dist, dev)
     attn_ms = [e[0].elapsed_time(e[1]) for e in evs]
     um_ms = [e[1].elapsed_time(e[2]) for e in evs]
     attn_avg_ms = max_over_ranks(sum(attn_ms) / len(attn_ms), dist, dev)
@@ -304,12 +313,11 @@ def run_gpu(args):
         abytes, prefix_bytes = attn_bytes(w, lens)
         n_masked = int(sets[0]["mask"].sum())
         ubytes = unmask_bytes(w, n_masked)
-        units = rows * args.steps * world
         achieved = abytes / (attn_avg_ms * 1e-3) / 1e9
         traffic = load_traffic(w)
         rec = {
             "metric": "denoise-step block-tokens/s",
-            "value": units / (ms * 1e-3),
+            "value": value,
             "unit": "block-tokens/s",
             "n_gpus": world,
             "steps": args.steps,
@@ -608,6 +616,8 @@ def main(argv=None):
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
     ap.add_argument("--workload", type=int, default=1, choices=[1, 2, 3, 4])
     ap.add_argument("--graph-steps", type=int, default=400)
+    ap.add_argument("--sets", type=int, default=4,
+                    help="rotating input sets (4 keep every step's inputs out of L2)")
     ap.add_argument("--e2e-steps", type=int, default=200)
     ap.add_argument("--cpu-seconds", type=float, default=10.0)
     ap.add_argument("--no-cpu-baseline", action="store_true")
