@@ -74,6 +74,19 @@ def test_small_cases_full(case):
     _full_check(inp, dtype)
 
 
+@pytest.mark.parametrize("dtype,H_kv,lens", [
+    # 64 near-equal pairs: one CTA per pair (no split, nothing to combine)
+    (torch.bfloat16, 8, [700, 690, 710, 705, 699, 701, 640, 720]),
+    (torch.float32, 4, [300] * 16),
+    # 64 pairs of very different lengths: balanced split + combine
+    (torch.bfloat16, 8, [100, 3000, 50, 2200, 900, 0, 1500, 4096]),
+])
+def test_pair_mode_and_split_mode(dtype, H_kv, lens):
+    w = _w(dtype, len(lens), 16, 4 * H_kv, H_kv, 128 if dtype == torch.bfloat16 else 64)
+    inp = workloads.attention_inputs(w, device=DEV, lens=lens)
+    _full_check(inp, dtype)
+
+
 def test_explicit_scale_and_padding_rows():
     w = _w(torch.bfloat16, 3, 16, 16, 4, 128)
     inp = workloads.attention_inputs(w, device=DEV, lens=[40, 0, 333], pad_rows=13)
