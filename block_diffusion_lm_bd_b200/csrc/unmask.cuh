@@ -38,6 +38,7 @@ struct UnmaskWs {
   int *n_masked;         // [1]
   int *rank;             // [rows]  rank among masked rows, -1 if unmasked
   UnmaskPart *row_part;  // [rows]  rows finished inside one CTA
+  int2 *row_meta;        // [rows]  (slot of the row's first record or -1 if whole, last CTA)
   UnmaskPart *slot;      // [G][2]  first / last cut segment of each CTA
 };
 
@@ -51,6 +52,8 @@ __host__ __device__ inline size_t unmask_ws_layout(int rows, int G, UnmaskWs *ws
   off = align256(off + sizeof(int) * size_t(rows));
   if (ws) ws->row_part = reinterpret_cast<UnmaskPart *>(base + off);
   off = align256(off + sizeof(UnmaskPart) * size_t(rows));
+  if (ws) ws->row_meta = reinterpret_cast<int2 *>(base + off);
+  off = align256(off + sizeof(int2) * size_t(rows));
   if (ws) ws->slot = reinterpret_cast<UnmaskPart *>(base + off);
   off = align256(off + sizeof(UnmaskPart) * size_t(G) * 2);
   return off;
@@ -259,10 +262,15 @@ __global__ void __launch_bounds__(kUnmaskThreads, kUnmaskCtasPerSm)
 
     UnmaskPart r = um_block_reduce(m, idx, s, sm_m, sm_i, sm_s);
     if (tid == 0) {
-      if (v0 == 0 && v1 == V)
+      const bool whole = (v0 == 0 && v1 == V);
+      const int slot = 2 * c + (rho == rho0 ? 0 : 1);
+      if (whole)
         p.ws.row_part[row] = r;
       else
-        p.ws.slot[2 * int64_t(c) + (rho == rho0 ? 0 : 1)] = r;
+        p.ws.slot[slot] = r;
+      // the CTA holding the row's first element describes where its records are
+      if (v0 == 0)
+        p.ws.row_meta[row] = whole ? make_int2(-1, c) : make_int2(slot, int(part_owner(rs + V - 1, W, G)));
     }
   }
 }
@@ -318,18 +326,26 @@ __global__ void __launch_bounds__(kUnmaskFinalizeThreads)
     s_commit[lr] = 0;
     s_conf[lr] = -1.0;
     if (!mk) continue;
-    const int64_t e0 = int64_t(p.ws.rank[r]) * V;
-    const int64_t c0 = part_owner(e0, W, G), c1 = part_owner(e0 + V - 1, W, G);
+    // where the row's records are (written by the CTA holding its first element)
+    const int2 meta = p.ws.row_meta[r];
     UnmaskPart a;
-    if (c0 == c1) {
+    if (meta.x < 0) {
       a = p.ws.row_part[r];
-    } else if (c1 - c0 < kDirectParts) {
-      a.m = -INFINITY;
-      a.sum = 0.0;
-      a.idx = INT_MAX;
+    } else if (W >= G && meta.y - meta.x / 2 < kDirectParts) {
+      // every CTA range is non-empty: CTA c > c0 holds its part in slot 2c
+      const int c0 = meta.x / 2, c1 = meta.y;
+      UnmaskPart q[kDirectParts];
 #pragma unroll
-      for (int k = 0; k < kDirectParts; ++k)
-        if (c0 + k <= c1) um_record_of(p, c0 + k, c0, e0, W, G, a);
+      for (int k = 0; k < kDirectParts; ++k) {
+        q[k].m = -INFINITY;
+        q[k].sum = 0.0;
+        q[k].idx = INT_MAX;
+        if (c0 + k <= c1) q[k] = p.ws.slot[k == 0 ? meta.x : 2 * (c0 + k)];
+      }
+      um_merge(q[0], q[1]);
+      um_merge(q[2], q[3]);
+      um_merge(q[0], q[2]);
+      a = q[0];
     } else {
       s_queue[atomicAdd(&s_nq, 1)] = lr;
       continue;
