@@ -160,3 +160,77 @@ def test_permutation_equivariance_on_gpu():
     o2, _ = _gpu(pin)
     err = float((o2 - o[:, perm]).abs().max() / o.std())
     assert err < 1e-2, err
+
+
+def _split_pair_inputs(step):
+    # 64 (b, kv) pairs of very different lengths: most pairs are split over
+    # several CTAs, so their parts are merged through the ticket words
+    w = _w(torch.bfloat16, 8, 16, 32, 8, 128)
+    return workloads.attention_inputs(w, device=DEV, step=step,
+                                      lens=[100, 3000, 50, 2200, 900, 0, 1500, 4096])
+
+
+def _oracle(inp):
+    return block_attention(inp["q"], inp["k_prefix"], inp["v_prefix"], inp["k_blk"], inp["v_blk"],
+                           inp["prefix_len_host"], inp["prefix_offset_host"])
+
+
+@pytest.mark.parametrize("fill", [0x00, 0xFF, "random"])
+def test_workspace_reuse_with_arbitrary_initial_contents(fill):
+    """The workspace needs no clearing: calls on a reused workspace whose
+    initial bytes are arbitrary all match the oracle."""
+    first = _split_pair_inputs(0)
+    B, S, H_q, d = first["q"].shape
+    nbytes = api.attn_workspace_bytes(B, S, H_q, first["k_blk"].shape[2], d)
+    if fill == "random":
+        ws = torch.randint(0, 256, (nbytes,), dtype=torch.uint8, device=DEV,
+                           generator=torch.Generator(device=DEV).manual_seed(11))
+    else:
+        ws = torch.full((nbytes,), fill, dtype=torch.uint8, device=DEV)
+    for step in range(3):
+        inp = first if step == 0 else _split_pair_inputs(step)
+        o, lse = api.attn_step(inp["q"], inp["k_prefix"], inp["v_prefix"], inp["k_blk"],
+                               inp["v_blk"], inp["prefix_len"], inp["prefix_offset"], workspace=ws)
+        torch.cuda.synchronize()
+        assert api.get_device_status() == 0
+        ro, rl = _oracle(inp)
+        err, raw = attn_err(to_np(o), ro)
+        assert err <= ATTN_TOL[torch.bfloat16], (step, err, raw)
+        assert float(np.abs(to_np(lse) - rl).max()) <= LSE_TOL[torch.bfloat16], step
+
+
+def test_cuda_graph_replays_match_oracle():
+    """A captured call replays with the same launch arguments every time; each
+    replay on new input values must still merge its split pairs correctly."""
+    inp = _split_pair_inputs(0)
+    B, S, H_q, d = inp["q"].shape
+    H_kv = inp["k_blk"].shape[2]
+    ws = torch.empty(api.attn_workspace_bytes(B, S, H_q, H_kv, d), dtype=torch.uint8, device=DEV)
+    o = torch.empty(B, S, H_q, d, device=DEV)
+    lse = torch.empty(B, H_q, S, device=DEV)
+    st = torch.cuda.Stream(DEV)
+
+    def call():
+        api.attn_step(inp["q"], inp["k_prefix"], inp["v_prefix"], inp["k_blk"], inp["v_blk"],
+                      inp["prefix_len"], inp["prefix_offset"], o=o, lse=lse, workspace=ws,
+                      stream=st)
+
+    with torch.cuda.stream(st):
+        call()
+    st.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=st):
+        call()
+    for step in range(1, 4):
+        new = _split_pair_inputs(step)
+        for k in ("q", "k_prefix", "v_prefix", "k_blk", "v_blk"):
+            inp[k].copy_(new[k])
+        torch.cuda.synchronize()
+        g.replay()
+        torch.cuda.synchronize()
+        assert api.get_device_status() == 0
+        ro, rl = _oracle(new)
+        err, raw = attn_err(to_np(o), ro)
+        assert err <= ATTN_TOL[torch.bfloat16], (step, err, raw)
+        assert float(np.abs(to_np(lse) - rl).max()) <= LSE_TOL[torch.bfloat16], step
+    del g
