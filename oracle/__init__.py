@@ -9,7 +9,9 @@ restatement of what the denoise step computes, written from the source pages:
   §Methodology > Generation process (Algorithm 1: S masked tokens refined over
   T steps, attending to the context-tower KV of past blocks and the current
   block's bidirectional KV), and §Training and conditioning > Sampling
-  (Algorithm 2: confidence unmasking with threshold gamma).
+  (Algorithm 2: confidence unmasking with threshold gamma), and the fourth
+  bullet of §Generation process (a committed block extends the prefix that the
+  next block attends to: the prefix-cache append).
 * "Training Hybrid Block Diffusion Language Models with Partial
   Bidirectionality" (gist.science, 2607.02805), §Methodology: the clean-prefix
   cache depends only on the prefix, never on the diffusion step, so the
@@ -30,6 +32,7 @@ hand-enumerated golden cases. Whole-pipeline numbers against the pages are
 from .attention import attend, block_attention, lse_combine
 from .unmask import confidence_unmask, top2_gap
 from .loop import block_loop
+from .kv_cache import kv_append
 
 __all__ = [
     "attend",
@@ -38,4 +41,5 @@ __all__ = [
     "confidence_unmask",
     "top2_gap",
     "block_loop",
+    "kv_append",
 ]

@@ -15,6 +15,7 @@ import os
 import pytest
 
 import test_oracle_attention as TA
+import test_oracle_kv_cache as TK
 import test_oracle_unmask as TU
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -106,6 +107,23 @@ def test_unmask_mutant_is_caught(mut, monkeypatch):
     assert _some_pin_fails(TU, patches, monkeypatch), f"no pin caught mutant {name!r}"
 
 
+KV_MUTANTS = [
+    ("append one row late", "lo = off[b] + L[b]\n", "lo = off[b] + L[b] + 1\n"),
+    ("length not advanced", "        L[b] += S\n", ""),
+    ("capacity not checked", "L[b] + S <= cap[b]", "True"),
+    ("mask ignored", "        if not sel[b]:\n            continue\n", ""),
+    ("K and V swapped", "        v[lo:lo + S] = vn[b]\n", "        v[lo:lo + S] = kn[b]\n"),
+]
+
+
+@pytest.mark.parametrize("mut", KV_MUTANTS, ids=[m[0] for m in KV_MUTANTS])
+def test_kv_append_mutant_is_caught(mut, monkeypatch):
+    name, old, new = mut
+    mod = _load_mutant("oracle/kv_cache.py", old, new, "mut_kv")
+    assert _some_pin_fails(TK, {"kv_append": mod.kv_append}, monkeypatch), \
+        f"no pin caught mutant {name!r}"
+
+
 def test_unmutated_copy_passes_every_pin(monkeypatch):
     """Control: the loader itself does not make pins fail."""
     mod = _load_mutant("oracle/attention.py", "import numpy as np", "import numpy as np", "same_attn")
@@ -115,3 +133,5 @@ def test_unmutated_copy_passes_every_pin(monkeypatch):
     mod = _load_mutant("oracle/unmask.py", "import numpy as np", "import numpy as np", "same_unmask")
     assert not _some_pin_fails(TU, {"confidence_unmask": mod.confidence_unmask,
                                     "top2_gap": mod.top2_gap}, monkeypatch)
+    mod = _load_mutant("oracle/kv_cache.py", "import numpy as np", "import numpy as np", "same_kv")
+    assert not _some_pin_fails(TK, {"kv_append": mod.kv_append}, monkeypatch)
