@@ -55,6 +55,8 @@ def _lib():
     lib.bd_unmask.argtypes = [vp, vp, f32, vp, vp, vp, vp, i32, i32, i32, i32, vp, sz, vp]
     lib.bd_unmask_noalloc.restype = i32
     lib.bd_unmask_noalloc.argtypes = [vp, vp, f32, vp, vp, vp, vp, i32, i32, i32, i32, vp]
+    lib.bd_kv_append.restype = i32
+    lib.bd_kv_append.argtypes = [vp, vp, i64, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, vp]
     lib.bd_get_device_status.restype = i32
     lib.bd_get_device_status.argtypes = [vp]
     lib.bd_debug_wait_timeout.restype = i32
@@ -180,6 +182,34 @@ def unmask(logits, mask, gamma, block_S=0, commit_at_least_one=False, tokens_out
         _ptr(workspace), workspace.numel() * workspace.element_size(), _stream_ptr(stream, dev))
     _check(st, "bd_unmask")
     return {"tokens": tokens_out, "conf": conf_out, "commit": commit_out, "mask_out": mask_out}
+
+
+def kv_append(k_prefix, v_prefix, k_new, v_new, prefix_len, prefix_offset, prefix_capacity,
+              seq_mask=None, stream=None):
+    """bd_kv_append on torch tensors: appends k_new / v_new [B,S,H_kv,d] after
+    each selected sequence's prefix rows and advances prefix_len in place."""
+    B, S, H_kv, d = k_new.shape
+    dev = k_new.device
+    if k_new.dtype not in _DTYPES:
+        raise ValueError(f"unsupported dtype {k_new.dtype}")
+    for t, nm in ((k_prefix, "k_prefix"), (v_prefix, "v_prefix"), (k_new, "k_new"),
+                  (v_new, "v_new")):
+        _need(t, nm, k_new.dtype, dev)
+    if k_prefix.shape[1:] != (H_kv, d) or v_prefix.shape != k_prefix.shape:
+        raise ValueError("k_prefix / v_prefix must be [rows, H_kv, d]")
+    if v_new.shape != k_new.shape:
+        raise ValueError("v_new must have the shape of k_new")
+    _need(prefix_len, "prefix_len", torch.int32, dev)
+    _need(prefix_offset, "prefix_offset", torch.int64, dev)
+    _need(prefix_capacity, "prefix_capacity", torch.int64, dev)
+    if seq_mask is not None:
+        _need(seq_mask, "seq_mask", torch.uint8, dev)
+    st = _lib().bd_kv_append(
+        _ptr(k_prefix), _ptr(v_prefix), int(k_prefix.shape[0]), _ptr(k_new), _ptr(v_new),
+        _ptr(prefix_len), _ptr(prefix_offset), _ptr(prefix_capacity), _ptr(seq_mask), B, S, H_kv,
+        d, _DTYPES[k_new.dtype], _stream_ptr(stream, dev))
+    _check(st, "bd_kv_append")
+    return prefix_len
 
 
 def unmask_noalloc(logits, mask, gamma, block_S=0, commit_at_least_one=False, tokens_out=None,

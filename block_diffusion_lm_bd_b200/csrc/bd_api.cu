@@ -10,6 +10,7 @@
 #include "attn_combine.cuh"
 #include "attn_simt.cuh"
 #include "attn_tc.cuh"
+#include "kv_append.cuh"
 #include "unmask.cuh"
 
 namespace {
@@ -242,6 +243,50 @@ bd_status bd_unmask(const float *logits, const uint8_t *mask, float gamma, int32
   fp.ws = rp.ws;
   const int grid = (rows + fp.rows_per_cta - 1) / fp.rows_per_cta;
   launch_pdl(bd::unmask_finalize_kernel, dim3(grid), dim3(bd::kUnmaskFinalizeThreads), 0, cs, fp);
+  return check_launch();
+}
+
+bd_status bd_kv_append(void *k_prefix, void *v_prefix, int64_t prefix_rows, const void *k_new,
+                       const void *v_new, int32_t *prefix_len, const int64_t *prefix_offset,
+                       const int64_t *prefix_capacity, const uint8_t *seq_mask, int B, int S,
+                       int H_kv, int d, bd_dtype dtype, bd_stream_t stream) {
+  if (B < 0 || B > bd::kMaxBatch || S < 1 || S > 64 || H_kv < 1 || H_kv > 64)
+    return BD_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return BD_ERR_UNSUPPORTED;
+  if (dtype != BD_DTYPE_F32 && dtype != BD_DTYPE_BF16) return BD_ERR_INVALID_ARG;
+  if (prefix_rows < 0 || prefix_rows > (int64_t(1) << 40)) return BD_ERR_INVALID_ARG;
+  if (B == 0) return BD_OK;
+  if (!k_prefix || !v_prefix || !k_new || !v_new || !prefix_len || !prefix_offset ||
+      !prefix_capacity)
+    return BD_ERR_INVALID_ARG;
+  if (!aligned16(k_prefix) || !aligned16(v_prefix) || !aligned16(k_new) || !aligned16(v_new) ||
+      (reinterpret_cast<uintptr_t>(prefix_len) & 3u) ||
+      (reinterpret_cast<uintptr_t>(prefix_offset) & 7u) ||
+      (reinterpret_cast<uintptr_t>(prefix_capacity) & 7u))
+    return BD_ERR_INVALID_ARG;
+  const int64_t row_bytes = int64_t(H_kv) * d * (dtype == BD_DTYPE_BF16 ? 2 : 4);
+  // the new K/V must not overlap the cache they are copied into
+  auto overlap = [](const void *a, int64_t na, const void *b, int64_t nb) {
+    const uintptr_t x = reinterpret_cast<uintptr_t>(a), y = reinterpret_cast<uintptr_t>(b);
+    return x < y + uintptr_t(nb) && y < x + uintptr_t(na);
+  };
+  const int64_t new_bytes = int64_t(B) * S * row_bytes, cache_bytes = prefix_rows * row_bytes;
+  for (const void *src : {k_new, v_new})
+    for (const void *dst : {static_cast<const void *>(k_prefix), static_cast<const void *>(v_prefix)})
+      if (overlap(src, new_bytes, dst, cache_bytes)) return BD_ERR_INVALID_ARG;
+  bd::KvAppendParams p = {};
+  p.k_prefix = static_cast<int4 *>(k_prefix);
+  p.v_prefix = static_cast<int4 *>(v_prefix);
+  p.prefix_rows = prefix_rows;
+  p.k_new = static_cast<const int4 *>(k_new);
+  p.v_new = static_cast<const int4 *>(v_new);
+  p.prefix_len = prefix_len;
+  p.prefix_offset = prefix_offset;
+  p.prefix_capacity = prefix_capacity;
+  p.seq_mask = seq_mask;
+  p.S = S;
+  p.row_vecs = row_bytes / 16;
+  bd::kv_append_kernel<<<B, bd::kAppendThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(p);
   return check_launch();
 }
 

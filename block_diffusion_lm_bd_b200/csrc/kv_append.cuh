@@ -1,0 +1,80 @@
+// Committing a finished block into the prefix cache ("Technical summary:
+// Nemotron-TwoTower", Methodology > Generation process, fourth bullet): the
+// clean K/V of the block's S tokens go after the sequence's old prefix rows,
+// and the sequence's prefix length grows by S.
+//
+// The S new rows of a sequence are contiguous in k_new (S * H_kv * d elements)
+// and land on S contiguous rows of the cache, so each of K and V is one
+// contiguous copy of S * H_kv * d * elem bytes (a multiple of 128 bytes for
+// d in {64, 128}). One CTA per sequence: it checks the bounds, copies with
+// 16-byte loads kept several deep in flight, and only then updates the
+// length, which no other CTA reads.
+#pragma once
+
+#include "bd_common.cuh"
+
+namespace bd {
+
+constexpr int kAppendThreads = 512;
+constexpr int kAppendUnroll = 8;
+
+struct KvAppendParams {
+  int4 *k_prefix;
+  int4 *v_prefix;
+  int64_t prefix_rows;
+  const int4 *k_new;
+  const int4 *v_new;
+  int32_t *prefix_len;
+  const int64_t *prefix_offset;
+  const int64_t *prefix_capacity;
+  const uint8_t *seq_mask;
+  int S;
+  int64_t row_vecs;  // 16-byte vectors per cache row (H_kv * d * elem / 16)
+};
+
+__global__ void __launch_bounds__(kAppendThreads) kv_append_kernel(KvAppendParams p) {
+  __shared__ int64_t s_dst;
+  __shared__ int s_len, s_go;
+  const int b = blockIdx.x;
+  if (threadIdx.x == 0) {
+    const bool sel = (p.seq_mask == nullptr) || (p.seq_mask[b] != 0);
+    const int64_t L = p.prefix_len[b], off = p.prefix_offset[b], cap = p.prefix_capacity[b];
+    const bool ok = L >= 0 && off >= 0 && cap >= 0 && L + p.S <= cap &&
+                    off + L + p.S <= p.prefix_rows && L + p.S <= INT32_MAX;
+    if (sel && !ok) record_status(BD_ERR_DEVICE_ARG);
+    s_go = (sel && ok) ? 1 : 0;
+    s_dst = off + L;
+    s_len = int(L);
+  }
+  __syncthreads();
+  if (!s_go) return;
+  const int64_t n = int64_t(p.S) * p.row_vecs;
+  const int4 *sk = p.k_new + int64_t(b) * n;
+  const int4 *sv = p.v_new + int64_t(b) * n;
+  int4 *dk = p.k_prefix + s_dst * p.row_vecs;
+  int4 *dv = p.v_prefix + s_dst * p.row_vecs;
+  constexpr int64_t step = int64_t(kAppendThreads) * kAppendUnroll;
+  for (int64_t i0 = threadIdx.x; i0 < n; i0 += step) {
+    int4 a[kAppendUnroll], c[kAppendUnroll];
+#pragma unroll
+    for (int k = 0; k < kAppendUnroll; ++k) {
+      const int64_t i = i0 + int64_t(k) * kAppendThreads;
+      if (i < n) {
+        a[k] = __ldcs(sk + i);
+        c[k] = __ldcs(sv + i);
+      }
+    }
+#pragma unroll
+    for (int k = 0; k < kAppendUnroll; ++k) {
+      const int64_t i = i0 + int64_t(k) * kAppendThreads;
+      if (i < n) {
+        dk[i] = a[k];
+        dv[i] = c[k];
+      }
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) p.prefix_len[b] = s_len + p.S;
+}
+
+}  // namespace bd

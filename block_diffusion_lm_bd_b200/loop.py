@@ -8,7 +8,10 @@ Algorithm 2) the positions whose confidence is higher than gamma. Committed
 tokens are final.
 
 Host orchestration only: every step is one bd_attn_step and one bd_unmask
-(mask updated in place, optional per-block fallback). Committed tokens
+(mask updated in place, optional per-block fallback); when the block is done,
+commit_block is one bd_kv_append: the block's clean K/V (the context tower's,
+supplied by the caller) join the prefix cache, so the next block's prefix is
+the old one followed by this block (Generation process, fourth bullet). Committed tokens
 accumulate in one tokens buffer because bd_unmask leaves the rows that are no
 longer masked untouched. The only synchronisation per step is the read-back
 of the mask (one byte per position) that decides whether to stop.
@@ -72,6 +75,14 @@ class BlockLoop:
         self.commit_step[newly] = t
         self.per_step.append(int(newly.sum()))
         return int(m.sum())
+
+    def commit_block(self, cache, k_clean, v_clean, prefix_capacity, seq_mask=None):
+        """Append the committed block's clean K/V [B,S,H_kv,d] to the prefix
+        cache in `cache` (k_prefix, v_prefix, prefix_len, prefix_offset);
+        prefix_len grows by S for every selected sequence."""
+        api.kv_append(cache["k_prefix"], cache["v_prefix"], k_clean, v_clean, cache["prefix_len"],
+                      cache["prefix_offset"], prefix_capacity, seq_mask=seq_mask,
+                      stream=self.stream)
 
     def run(self, step_inputs, T):
         """Run up to T steps; stop when every position is committed."""

@@ -52,7 +52,7 @@ typedef enum {
   BD_ERR_UNSUPPORTED = 2, /* valid, but outside what the kernels implement  */
   BD_ERR_CUDA = 3,        /* a CUDA runtime / driver call or launch failed  */
   BD_ERR_TIMEOUT = 4,     /* device: a bounded wait ran out (kernel exited) */
-  BD_ERR_DEVICE_ARG = 5   /* device: prefix_len / prefix_offset out of range */
+  BD_ERR_DEVICE_ARG = 5   /* device: a length / offset / capacity out of range */
 } bd_status;
 
 typedef enum { BD_DTYPE_F32 = 0, BD_DTYPE_BF16 = 1 } bd_dtype;
@@ -182,6 +182,48 @@ bd_status bd_unmask_noalloc(const float *logits, const uint8_t *mask, float gamm
                             int32_t *tokens_out, float *conf_out, uint8_t *commit_out,
                             uint8_t *mask_out, int rows, int V, int block_S,
                             int commit_at_least_one, bd_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Committing a finished block into the prefix cache                        */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Appends the clean K/V of a committed block to the prefix cache
+ * ("Technical summary: Nemotron-TwoTower", Methodology > Generation process,
+ * fourth bullet: once a block is committed, the context tower takes its clean
+ * tokens into its state, and the next block attends to them as prefix). The
+ * caller supplies those K/V (the context tower's keys and values of the
+ * block's committed tokens); this call places them.
+ *
+ * For every sequence b with seq_mask == NULL or seq_mask[b] != 0:
+ *     rows prefix_offset[b] + prefix_len[b] + i, i = 0 .. S-1, of k_prefix
+ *     and v_prefix  <-  k_new[b, i, :, :] and v_new[b, i, :, :]
+ *     prefix_len[b] += S
+ * so the next bd_attn_step of sequence b sees the block's S keys after its
+ * old prefix. Other rows and the other sequences' lengths are not touched.
+ *
+ * Arguments (all device pointers unless said otherwise):
+ *   k_prefix, v_prefix [prefix_rows, H_kv, d] dtype   WRITTEN (appended rows)
+ *   prefix_rows   rows allocated in k_prefix / v_prefix (host int)
+ *   k_new, v_new  [B, S, H_kv, d] dtype               read
+ *   prefix_len    int32 [B]                            READ AND WRITTEN
+ *   prefix_offset int64 [B]: first row of sequence b   read
+ *   prefix_capacity int64 [B]: rows reserved for sequence b from its
+ *                 offset (its appends must stay inside them)   read
+ *   seq_mask      uint8 [B], or NULL for every sequence    read
+ * Supported: d in {64, 128}; 1 <= S <= 64; 1 <= H_kv <= 64; B <= 4096;
+ * k_new / v_new must not overlap the cache. Otherwise BD_ERR_INVALID_ARG /
+ * BD_ERR_UNSUPPORTED, and nothing is launched. A selected sequence whose new
+ * rows would leave [offset, offset + capacity) or [0, prefix_rows), or whose
+ * length, offset or capacity is negative, is skipped (nothing of it is
+ * written, its length is unchanged) and the device status becomes
+ * BD_ERR_DEVICE_ARG. One CTA per sequence does the copy and then the length
+ * update, so no other thread reads a length while it changes.
+ */
+bd_status bd_kv_append(void *k_prefix, void *v_prefix, int64_t prefix_rows, const void *k_new,
+                       const void *v_new, int32_t *prefix_len, const int64_t *prefix_offset,
+                       const int64_t *prefix_capacity, const uint8_t *seq_mask, int B, int S,
+                       int H_kv, int d, bd_dtype dtype, bd_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
 /* Status, diagnostics                                                      */

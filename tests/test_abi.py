@@ -32,7 +32,8 @@ def declared_functions():
 def test_header_declares_the_boundary():
     names = declared_functions()
     for required in ("bd_attn_step", "bd_attn_workspace_bytes", "bd_unmask",
-                     "bd_unmask_workspace_bytes", "bd_get_device_status", "bd_status_string"):
+                     "bd_unmask_workspace_bytes", "bd_get_device_status", "bd_status_string",
+                     "bd_kv_append"):
         assert required in names
 
 
@@ -144,3 +145,40 @@ def test_product_package_never_imports_the_oracle():
                 src = open(os.path.join(dirpath, f)).read()
                 assert not re.search(r"^\s*(from|import)\s+oracle\b", src, re.M), f
                 assert "oracle/" not in src, f
+
+
+def _append(lib, **kw):
+    a = dict(kp=1 << 20, vp=2 << 20, rows=100, kn=3 << 20, vn=4 << 20, pl=16, po=16, pc=16, sm=0,
+             B=2, S=16, Hkv=2, d=64, dtype=1, st=0)
+    a.update(kw)
+    vp = lambda x: ctypes.c_void_p(x) if x else None
+    return lib.bd_kv_append(vp(a["kp"]), vp(a["vp"]), a["rows"], vp(a["kn"]), vp(a["vn"]),
+                            vp(a["pl"]), vp(a["po"]), vp(a["pc"]), vp(a["sm"]), a["B"], a["S"],
+                            a["Hkv"], a["d"], a["dtype"], vp(a["st"]))
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(d=96), UNSUPPORTED),
+    (dict(S=0), INVALID),
+    (dict(S=65), INVALID),
+    (dict(Hkv=0), INVALID),
+    (dict(B=-1), INVALID),
+    (dict(B=5000), INVALID),
+    (dict(dtype=7), INVALID),
+    (dict(rows=-1), INVALID),
+    (dict(kp=0), INVALID),
+    (dict(kn=0), INVALID),
+    (dict(pl=0), INVALID),
+    (dict(pc=0), INVALID),
+    (dict(kp=(1 << 20) + 8), INVALID),            # misaligned cache
+    (dict(pl=18), INVALID),                       # int32 array misaligned
+    (dict(pc=20), INVALID),                       # int64 array misaligned
+    (dict(kn=(1 << 20) + 4096), INVALID),         # new K inside the K cache
+    (dict(vn=(2 << 20)), INVALID),                # new V is the V cache itself
+])
+def test_kv_append_host_validation(lib, kw, code):
+    assert _append(lib, **kw) == code
+
+
+def test_kv_append_empty_batch_is_a_no_op(lib):
+    assert _append(lib, B=0) == 0

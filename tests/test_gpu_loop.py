@@ -88,3 +88,27 @@ def test_full_size_loop_invariants_and_first_steps():
     assert (loop.commit_step >= 0).all()
     print(f"loop: {steps} steps, committed per step {loop.per_step}, "
           f"tokens per step {w.B * w.S / steps:.1f}")
+
+
+def test_commit_block_appends_to_the_prefix_cache():
+    """Algorithm 1's tail: after the loop, the block's clean K/V join the prefix
+    cache (bit-exact against the oracle); the next step's attention then reads
+    a prefix longer by S."""
+    from oracle.kv_cache import kv_append
+
+    w = workloads.WORKLOADS[4].with_(B=4, prefix_len=200, V=4096)
+    base = workloads.attention_inputs(w, device=DEV, pad_rows=w.S)
+    cap = (base["prefix_offset"][1:] - base["prefix_offset"][:-1]).contiguous()
+    loop = BlockLoop(w.B, w.S, w.H_q, w.H_kv, w.d, w.V, w.gamma, DEV, commit_at_least_one=True)
+    steps = loop.run(lambda t: _inputs(w, t, base), w.steps)
+    assert steps <= w.S and not loop.mask.any()
+    g = torch.Generator(device=DEV).manual_seed(77)
+    kc = torch.randn(w.B, w.S, w.H_kv, w.d, device=DEV, generator=g).to(w.dtype)
+    vc = torch.randn(w.B, w.S, w.H_kv, w.d, device=DEV, generator=g).to(w.dtype)
+    ref = kv_append(base["k_prefix"], base["v_prefix"], kc, vc, base["prefix_len"],
+                    base["prefix_offset"][:w.B], cap)
+    loop.commit_block(base, kc, vc, cap)
+    torch.cuda.synchronize()
+    assert (base["k_prefix"].cpu().view(torch.int16).numpy() == ref[0]).all()
+    assert (base["v_prefix"].cpu().view(torch.int16).numpy() == ref[1]).all()
+    assert base["prefix_len"].cpu().tolist() == [200 + w.S] * w.B
