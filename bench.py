@@ -48,9 +48,14 @@ PROFILE_FILE = os.path.join(ROOT, "profiles", "attn_traffic.json")
 CSRC = os.path.join(ROOT, "block_diffusion_lm_bd_b200", "csrc")
 
 
+# the sources of the attention call's kernels: the DRAM traffic recorded in
+# profiles/attn_traffic.json is valid while these are unchanged
+ATTN_SOURCES = ("attn_combine.cuh", "attn_common.cuh", "attn_tc.cuh", "bd_common.cuh", "tc_ptx.cuh")
+
+
 def kernel_source_hash():
     h = hashlib.sha256()
-    for f in sorted(os.listdir(CSRC)):
+    for f in ATTN_SOURCES:
         with open(os.path.join(CSRC, f), "rb") as fh:
             h.update(f.encode() + fh.read())
     return h.hexdigest()[:16]
@@ -255,16 +260,25 @@ def run_gpu(args):
     stream.synchronize()
     assert api.get_device_status(stream) == 0
 
+    # The timed graph holds the steps only. A second graph of the same steps
+    # with event records around each call gives the attention / unmask split
+    # (event nodes between the kernels cost time of their own, so they stay
+    # out of the timed region).
     P = min(args.steps, args.graph_steps)
     n_full, tail = divmod(args.steps, P)
-    evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)]
-           for _ in range(P)]
     l0 = api.launch_count()
     g_main = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g_main, stream=stream):
         for i in range(P):
-            step(i, evs[i])
+            step(i)
     launches_per_step = (api.launch_count() - l0) / P
+    P_ev = min(P, 200)
+    evs = [[torch.cuda.Event(enable_timing=True, external=True) for _ in range(3)]
+           for _ in range(P_ev)]
+    g_ev = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_ev, stream=stream):
+        for i in range(P_ev):
+            step(i, evs[i])
     g_tail = None
     if tail:
         g_tail = torch.cuda.CUDAGraph()
@@ -291,10 +305,13 @@ def run_gpu(args):
             t1.record(stream)
         torch.cuda.synchronize(dev)
         barrier(dist, dev)
+    ms_local = t0.elapsed_time(t1)
+    for _ in range(2):
+        g_ev.replay()
+    torch.cuda.synchronize(dev)
     st = api.get_device_status(stream)
     if st != 0:
         raise RuntimeError(f"device status {api.status_string(st)}")
-    ms_local = t0.elapsed_time(t1)
     value, ms = aggregate_throughput(rows * args.steps, ms_local, dist, dev)
     attn_ms = [e[0].elapsed_time(e[1]) for e in evs]
     um_ms = [e[1].elapsed_time(e[2]) for e in evs]
@@ -365,9 +382,12 @@ def run_gpu(args):
 def run_loop(args):
     """The block refinement loop (workload 4): up to T denoise steps of B blocks,
     each step one bd_attn_step and one bd_unmask (fallback on, mask updated in
-    place), stopping when every block is committed. The T steps' inputs are
-    drawn before timing (q / block K,V / logits of step t from seed(t)); the
-    timed region is whole loops, including the per-step mask read-back."""
+    place), stopping when every block is committed, then the commit of the
+    block into the prefix cache (bd_kv_append of the block's clean K/V). The T
+    steps' inputs and the clean K/V are drawn before timing (q / block K,V /
+    logits of step t from seed(t)); the timed region is whole loops, including
+    the per-step mask read-back and the reset of the prefix lengths (a 256-byte
+    device copy) that lets every loop start from the same prefix."""
     from block_diffusion_lm_bd_b200 import api, build as _build, workloads
     from block_diffusion_lm_bd_b200.loop import BlockLoop
 
@@ -380,7 +400,15 @@ def run_loop(args):
     barrier(dist, dev)
     w = workloads.WORKLOADS[4]
     T = w.steps
-    base = workloads.attention_inputs(w, device=dev, step=1000 * rank)
+    # spare rows after every sequence: room for the committed block (and for
+    # the N_APPEND back-to-back commits timed on their own below)
+    N_APPEND = 20
+    base = workloads.attention_inputs(w, device=dev, step=1000 * rank, pad_rows=w.S * N_APPEND)
+    cap = (base["prefix_offset"][1:] - base["prefix_offset"][:-1]).contiguous()
+    plen0 = base["prefix_len"].clone()
+    cgen = torch.Generator(device=dev).manual_seed(w.seed(1000 * rank) + 900)
+    k_clean = (torch.randn((w.B, w.S, w.H_kv, w.d), generator=cgen, device=dev) * w.qkv_std).to(w.dtype)
+    v_clean = (torch.randn((w.B, w.S, w.H_kv, w.d), generator=cgen, device=dev) * w.qkv_std).to(w.dtype)
     steps_in = []
     for t in range(T):
         inp = dict(base)
@@ -390,10 +418,16 @@ def run_loop(args):
     stream = torch.cuda.Stream(device=dev)
     loop = BlockLoop(w.B, w.S, w.H_q, w.H_kv, w.d, w.V, w.gamma, dev, commit_at_least_one=True,
                      stream=stream)
+    def one_block():
+        base["prefix_len"].copy_(plen0, non_blocking=True)
+        loop.reset()
+        n = loop.run(lambda t: steps_in[t], T)
+        loop.commit_block(base, k_clean, v_clean, cap)
+        return n
+
     with torch.cuda.stream(stream):
         for _ in range(max(1, args.warmup // 10)):
-            loop.reset()
-            loop.run(lambda t: steps_in[t], T)
+            one_block()
     nloops = max(1, args.steps // 100)
     a = torch.cuda.Event(enable_timing=True)
     b = torch.cuda.Event(enable_timing=True)
@@ -406,14 +440,33 @@ def run_loop(args):
         with torch.cuda.stream(stream):
             a.record(stream)
             for _ in range(nloops):
-                loop.reset()
-                total_steps += loop.run(lambda t: steps_in[t], T)
+                total_steps += one_block()
             b.record(stream)
         torch.cuda.synchronize(dev)
         barrier(dist, dev)
     launches = api.launch_count() - l0
     ms = max_over_ranks(a.elapsed_time(b), dist, dev)
     assert api.get_device_status(stream) == 0
+    assert base["prefix_len"].cpu().tolist() == (plen0 + w.S).cpu().tolist()
+    # the commit alone: a CUDA graph of N_APPEND back-to-back bd_kv_append calls
+    # (each appends one more block), CUDA events around a replay
+    g_app = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g_app, stream=stream):
+        for _ in range(N_APPEND):
+            loop.commit_block(base, k_clean, v_clean, cap)
+    app_us = None
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            base["prefix_len"].copy_(plen0, non_blocking=True)
+            a.record(stream)
+            g_app.replay()
+            b.record(stream)
+            b.synchronize()
+            app_us = a.elapsed_time(b) * 1e3 / N_APPEND
+    torch.cuda.synchronize(dev)
+    assert api.get_device_status(stream) == 0
+    assert base["prefix_len"].cpu().tolist() == (plen0 + w.S * N_APPEND).cpu().tolist()
+    app_bytes = 2 * 2 * k_clean.numel() * k_clean.element_size()  # K and V, read + written
     if rank == 0:
         lens = base["prefix_len_host"].tolist()
         abytes, prefix_bytes = attn_bytes(w, lens)
@@ -438,6 +491,9 @@ def run_loop(args):
                        "parallelism": f"replicas x{world}"},
             "roofline": {"bound": "hbm", "prefix_kv_bytes_per_step": prefix_bytes,
                          "attn_bytes_per_step": abytes},
+            "kv_append": {"us_per_call": app_us, "bytes_per_call": app_bytes,
+                          "achieved_gbs": app_bytes / (app_us * 1e3),
+                          "note": "block commit (bd_kv_append), graph of back-to-back calls"},
             "gpu_launches": launches,
             "clocks": sampler.summary(),
             "kernel_source": kernel_source_hash(),
