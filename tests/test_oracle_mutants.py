@@ -16,6 +16,7 @@ import pytest
 
 import test_oracle_attention as TA
 import test_oracle_kv_cache as TK
+import test_oracle_lmhead as TL
 import test_oracle_unmask as TU
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -122,6 +123,29 @@ def test_kv_append_mutant_is_caught(mut, monkeypatch):
     mod = _load_mutant("oracle/kv_cache.py", old, new, "mut_kv")
     assert _some_pin_fails(TK, {"kv_append": mod.kv_append}, monkeypatch), \
         f"no pin caught mutant {name!r}"
+
+
+LMHEAD_MUTANTS = [
+    ("head not transposed", "return h @ _f64(w_vocab).T", "return h @ _f64(w_vocab)"),
+    ("row list ignored", "        h = h[np.asarray(rows, dtype=np.int64)]\n", "        pass\n"),
+    ("hidden scaled by 1/sqrt(D)", "return h @ _f64(w_vocab).T", "return (h @ _f64(w_vocab).T) / np.sqrt(h.shape[1])"),
+    ("unmasked rows predicted", "    idx = np.flatnonzero(m)\n", "    idx = np.arange(m.shape[0])\n"),
+]
+
+
+@pytest.mark.parametrize("mut", LMHEAD_MUTANTS, ids=[m[0] for m in LMHEAD_MUTANTS])
+def test_lmhead_mutant_is_caught(mut, monkeypatch):
+    name, old, new = mut
+    src = open(os.path.join(ROOT, "oracle/lmhead.py")).read()
+    assert src.count(old) >= 1, old
+    # the module imports confidence_unmask relatively: load it inside the package
+    import oracle
+    spec = importlib.util.spec_from_loader("oracle._mut_lmhead", loader=None)
+    mod = importlib.util.module_from_spec(spec)
+    mod.__package__ = "oracle"
+    exec(compile(src.replace(old, new), "<mutant lmhead>", "exec"), mod.__dict__)
+    patches = {"lmhead_logits": mod.lmhead_logits, "lmhead_unmask": mod.lmhead_unmask}
+    assert _some_pin_fails(TL, patches, monkeypatch), f"no pin caught mutant {name!r}"
 
 
 def test_unmutated_copy_passes_every_pin(monkeypatch):
