@@ -3,7 +3,7 @@
 confidence unmasking) on B200, printing one JSON line.
 
     python bench.py [--gpus N] [--steps K] [--warmup W] [--impl reference]
-                    [--workload 1]
+                    [--workload 1|2|3|4|5]
 
 Default workload: the bf16 decode step (B=8 sequences, H_q=32, H_kv=8,
 d=128, prefix 4096, block S=16, V=131072, gamma=0.9), synthetic data.
@@ -21,6 +21,10 @@ d=128, prefix 4096, block S=16, V=131072, gamma=0.9), synthetic data.
   cache is resident state in HBM.
 * cpu_baseline: the float64 oracle on a bounded sample, host cores.
 * --impl reference: the oracle as the reference arm.
+* --workload 2 / 3: ragged S=32 prefixes / one 262144-token prefix; 4: the
+  block loop (up to 16 steps of B=64 blocks, then the block commit into the
+  prefix cache); 5: the LM head fused with unmasking (128 rows, D=4096,
+  V=131072).
 Under torchrun (N > 1) every rank runs an independent replica (replicas
 only: the step has no exchange); the time is the max over ranks.
 """
@@ -624,6 +628,205 @@ def run_cpu_baseline(w, seconds):
             "host_cpus": len(os.sched_getaffinity(0))}
 
 
+# --------------------------------------------------------------------------
+# LM head fused with unmasking (workload 5)
+# --------------------------------------------------------------------------
+LMHEAD_CHUNK = 4096  # vocabulary tokens per oracle unit
+
+
+def lmhead_oracle_unit(h, W, mask, gamma):
+    """The oracle on one row against one LMHEAD_CHUNK-token slice of a head of
+    the workload's law: 1/(V/LMHEAD_CHUNK) of one row's projection + unmask."""
+    from oracle.lmhead import lmhead_unmask
+
+    lmhead_unmask(h, W, mask, gamma)
+
+
+def lmhead_cpu_sample(w, seconds):
+    from block_diffusion_lm_bd_b200 import workloads
+
+    D = w.extra["D"]
+    h, W = workloads.lmhead_inputs(w, device="cpu", rows=2, D=D, V=LMHEAD_CHUNK)
+    mask = np.ones(1, dtype=np.uint8)
+    per_unit = LMHEAD_CHUNK / w.V
+    t, n = 0.0, 0
+    while t < seconds:
+        t0 = time.perf_counter()
+        lmhead_oracle_unit(h[n % 2:n % 2 + 1], W, mask, w.gamma)
+        t += time.perf_counter() - t0
+        n += 1
+    return n * per_unit / t, n, t
+
+
+def _lmhead_sample_text(w, n, t):
+    return (f"{n} units in {t:.1f} s; one row's hidden state (D={w.extra['D']}) against a "
+            f"{LMHEAD_CHUNK}-token head of the same law per unit = 1/{w.V // LMHEAD_CHUNK} of one "
+            "row's projection + unmask, float64 NumPy")
+
+
+def run_lmhead(args):
+    """LM head fused with confidence unmasking at the decode step (workload 5):
+    the 128 masked rows' hidden states (D=4096) against a 131072-token bf16
+    head, one bd_lmhead_unmask call per step. The head (1 GiB) is larger than
+    L2, so every call streams it from HBM."""
+    from block_diffusion_lm_bd_b200 import api, build as _build, workloads
+
+    world, rank, local = dist_env()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    dist = init_dist(world, "nccl")
+    if rank == 0 and _build.needs_build():
+        _build.build()
+    barrier(dist, dev)
+    w = workloads.WORKLOADS[5]
+    rows, D, V = w.B * w.S, w.extra["D"], w.V
+    h, W = workloads.lmhead_inputs(w, device=dev, step=1000 * rank)
+    mask = torch.ones(rows, dtype=torch.uint8, device=dev)
+    ws = torch.empty(api.lmhead_unmask_workspace_bytes(rows, V, D), dtype=torch.uint8, device=dev)
+    tok = torch.empty(rows, dtype=torch.int32, device=dev)
+    conf = torch.empty(rows, dtype=torch.float32, device=dev)
+    com = torch.empty(rows, dtype=torch.uint8, device=dev)
+    stream = torch.cuda.Stream(device=dev)
+
+    def call():
+        api.lmhead_unmask(h, W, mask, w.gamma, tokens_out=tok, conf_out=conf, commit_out=com,
+                          workspace=ws, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(max(args.warmup, 3)):
+            call()
+    stream.synchronize()
+    assert api.get_device_status(stream) == 0
+    P = min(args.steps, 100)
+    n_full, tail = divmod(args.steps, P)
+    l0 = api.launch_count()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for _ in range(P):
+            call()
+    launches_per_call = (api.launch_count() - l0) / P
+    g_tail = None
+    if tail:
+        g_tail = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_tail, stream=stream):
+            for _ in range(tail):
+                call()
+    g.replay()
+    torch.cuda.synchronize(dev)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(dev)
+    with sampler:
+        barrier(dist, dev)
+        torch.cuda.synchronize(dev)
+        with torch.cuda.stream(stream):
+            t0.record(stream)
+            for _ in range(n_full):
+                g.replay()
+            if g_tail is not None:
+                g_tail.replay()
+            t1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(dist, dev)
+    st = api.get_device_status(stream)
+    if st != 0:
+        raise RuntimeError(f"device status {api.status_string(st)}")
+    value, ms = aggregate_throughput(rows * args.steps, t0.elapsed_time(t1), dist, dev)
+    call_us = ms * 1e3 / args.steps
+
+    # the same result unfused, for context: cuBLAS bf16 GEMM to bf16 logits,
+    # upcast to fp32, then bd_unmask
+    logits = torch.empty((rows, V), dtype=torch.float32, device=dev)
+    wsu = torch.empty(api.unmask_workspace_bytes(rows, V), dtype=torch.uint8, device=dev)
+
+    def unfused():
+        logits.copy_(torch.nn.functional.linear(h, W))
+        api.unmask(logits, mask, w.gamma, tokens_out=tok, conf_out=conf, commit_out=com,
+                   workspace=wsu, stream=stream)
+
+    with torch.cuda.stream(stream):
+        for _ in range(3):
+            unfused()
+        torch.cuda.synchronize(dev)
+        t0.record(stream)
+        for _ in range(20):
+            unfused()
+        t1.record(stream)
+    torch.cuda.synchronize(dev)
+    unfused_us = t0.elapsed_time(t1) * 1e3 / 20
+
+    # e2e: hidden states and mask from pinned host memory in, results out
+    h_host = h.to("cpu").pin_memory()
+    m_host = mask.to("cpu").pin_memory()
+    res_host = [torch.empty(t.shape, dtype=t.dtype).pin_memory() for t in (tok, conf, com)]
+    K = min(args.steps, args.e2e_steps)
+    with torch.cuda.stream(stream):
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        barrier(dist, dev)
+        a.record(stream)
+        for _ in range(K):
+            h.copy_(h_host, non_blocking=True)
+            mask.copy_(m_host, non_blocking=True)
+            call()
+            for dst, src in zip(res_host, (tok, conf, com)):
+                dst.copy_(src, non_blocking=True)
+        b.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(a.elapsed_time(b), dist, dev)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, n, t = lmhead_cpu_sample(w, args.cpu_seconds)
+        cpu = {"value": v, "unit": "block-tokens/s", "cores": cpu_threads(), "kind": "oracle",
+               "sample": _lmhead_sample_text(w, n, t), "host_cpus": len(os.sched_getaffinity(0))}
+    if rank == 0:
+        peak, peak_kind = hbm_peak()
+        hbm_bytes = V * D * 2 + rows * D * 2 + rows * 9
+        flops = 2.0 * rows * V * D
+        achieved = hbm_bytes / (call_us * 1e3)
+        try:
+            with open(PEAKS_FILE) as f:
+                tpeak = float(json.load(f)["bf16_tflops"])
+        except Exception:
+            tpeak = 1590.0
+        rec = {
+            "metric": "LM head + unmask block-tokens/s",
+            "value": value,
+            "unit": "block-tokens/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": ms / args.steps,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16",
+            "data": "synthetic (seeded; hidden states N(0,1), head of the decode step's logit law)",
+            "config": {"workload": f"LM head + unmask: {rows} masked rows, D={D}, V={V}, "
+                                   "bf16 head 1 GiB (> L2: streamed from HBM every call)",
+                       "parallelism": f"replicas x{world}"},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": None, "peak_kind": peak_kind,
+                         "kernel": "bd_lmhead_unmask (gather + tcgen05 projection/fold + finalize)",
+                         "algorithmic_bytes": hbm_bytes, "avg_call_us": call_us,
+                         "tensor_tflops": flops / (call_us * 1e-6) / 1e12,
+                         "tensor_frac_of_bf16_peak": flops / (call_us * 1e-6) / 1e12 / tpeak},
+            "unfused_context": {"us_per_call": unfused_us,
+                                "what": "torch bf16 GEMM to logits + fp32 upcast + bd_unmask"},
+            "cpu_baseline": cpu,
+            "e2e": {"value": rows * K * world / (e2e_ms * 1e-3), "unit": "block-tokens/s",
+                    "h2d_bytes_per_step": h_host.numel() * 2 + m_host.numel(),
+                    "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in res_host),
+                    "steps": K, "ms_per_step": e2e_ms / K},
+            "gpu_launches": int(round(launches_per_call * args.steps)),
+            "clocks": sampler.summary(),
+        }
+        print(json.dumps(rec))
+    if dist is not None:
+        dist.destroy_process_group()
+
+
 def run_reference(args):
     world, rank, _ = dist_env()
     if rank != 0:
@@ -631,6 +834,20 @@ def run_reference(args):
     from block_diffusion_lm_bd_b200 import workloads
 
     w = workloads.WORKLOADS[args.workload]
+    if args.workload == 5:
+        v, n, t = lmhead_cpu_sample(w, max(1.0, min(30.0, args.steps * 0.5)))
+        rec = {"impl": "reference", "metric": "LM head + unmask block-tokens/s", "value": v,
+               "unit": "block-tokens/s", "n_gpus": world, "steps": args.steps,
+               "warmup": args.warmup, "ms_per_step": t / max(n, 1) * 1e3,
+               "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+               "data": "synthetic (seeded)", "config": {"workload": workload_label(w),
+                                                        "parallelism": "host cores"},
+               "cpu_baseline": {"value": v, "unit": "block-tokens/s", "cores": cpu_threads(),
+                                "kind": "oracle", "sample": _lmhead_sample_text(w, n, t)},
+               "e2e": {"value": v, "unit": "block-tokens/s", "h2d_bytes_per_step": 0,
+                       "d2h_bytes_per_step": 0}}
+        print(json.dumps(rec))
+        return
     cache = [oracle_unit_inputs(w, s) for s in range(min(w.B, 2))]
     for i in range(args.warmup):
         oracle_unit(*cache[i % len(cache)], i % w.H_kv)
@@ -670,7 +887,7 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=4000)
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
-    ap.add_argument("--workload", type=int, default=1, choices=[1, 2, 3, 4])
+    ap.add_argument("--workload", type=int, default=1, choices=[1, 2, 3, 4, 5])
     ap.add_argument("--graph-steps", type=int, default=400)
     ap.add_argument("--sets", type=int, default=4,
                     help="rotating input sets (4 keep every step's inputs out of L2)")
@@ -684,6 +901,8 @@ def main(argv=None):
         run_reference(args)
     elif args.workload == 4:
         run_loop(args)
+    elif args.workload == 5:
+        run_lmhead(args)
     else:
         run_gpu(args)
 

@@ -55,6 +55,11 @@ def _lib():
     lib.bd_unmask.argtypes = [vp, vp, f32, vp, vp, vp, vp, i32, i32, i32, i32, vp, sz, vp]
     lib.bd_unmask_noalloc.restype = i32
     lib.bd_unmask_noalloc.argtypes = [vp, vp, f32, vp, vp, vp, vp, i32, i32, i32, i32, vp]
+    lib.bd_lmhead_unmask_workspace_bytes.restype = sz
+    lib.bd_lmhead_unmask_workspace_bytes.argtypes = [i32, i32, i32]
+    lib.bd_lmhead_unmask.restype = i32
+    lib.bd_lmhead_unmask.argtypes = [vp, vp, vp, f32, vp, vp, vp, vp, i32, i32, i32, i32, i32, vp,
+                                     sz, vp]
     lib.bd_kv_append.restype = i32
     lib.bd_kv_append.argtypes = [vp, vp, i64, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, vp]
     lib.bd_get_device_status.restype = i32
@@ -181,6 +186,42 @@ def unmask(logits, mask, gamma, block_S=0, commit_at_least_one=False, tokens_out
         _ptr(commit_out), _ptr(mask_out), rows, V, int(block_S), 1 if commit_at_least_one else 0,
         _ptr(workspace), workspace.numel() * workspace.element_size(), _stream_ptr(stream, dev))
     _check(st, "bd_unmask")
+    return {"tokens": tokens_out, "conf": conf_out, "commit": commit_out, "mask_out": mask_out}
+
+
+def lmhead_unmask_workspace_bytes(rows, V, D):
+    return int(_lib().bd_lmhead_unmask_workspace_bytes(rows, V, D))
+
+
+def lmhead_unmask(hidden, w_vocab, mask, gamma, block_S=0, commit_at_least_one=False,
+                  tokens_out=None, conf_out=None, commit_out=None, mask_out=None, workspace=None,
+                  stream=None):
+    """bd_lmhead_unmask on torch tensors: hidden bf16 [rows, D], w_vocab bf16
+    [V, D], mask uint8 [rows]. Returns the same dict as unmask()."""
+    rows, D = hidden.shape
+    V = w_vocab.shape[0]
+    dev = hidden.device
+    _need(hidden, "hidden", torch.bfloat16, dev)
+    _need(w_vocab, "w_vocab", torch.bfloat16, dev)
+    if w_vocab.shape[1] != D:
+        raise ValueError("w_vocab must be [V, D] with the hidden size D")
+    _need(mask, "mask", torch.uint8, dev)
+    if tokens_out is None:
+        tokens_out = torch.full((rows,), -1, dtype=torch.int32, device=dev)
+    if conf_out is None:
+        conf_out = torch.full((rows,), float("nan"), dtype=torch.float32, device=dev)
+    if commit_out is None:
+        commit_out = torch.empty(rows, dtype=torch.uint8, device=dev)
+    if workspace is None:
+        nbytes = lmhead_unmask_workspace_bytes(rows, V, D)
+        if nbytes == 0:
+            raise BdError(2, "bd_lmhead_unmask_workspace_bytes")
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    st = _lib().bd_lmhead_unmask(
+        _ptr(hidden), _ptr(w_vocab), _ptr(mask), float(gamma), _ptr(tokens_out), _ptr(conf_out),
+        _ptr(commit_out), _ptr(mask_out), rows, V, D, int(block_S), int(bool(commit_at_least_one)),
+        _ptr(workspace), workspace.numel() * workspace.element_size(), _stream_ptr(stream, dev))
+    _check(st, "bd_lmhead_unmask")
     return {"tokens": tokens_out, "conf": conf_out, "commit": commit_out, "mask_out": mask_out}
 
 

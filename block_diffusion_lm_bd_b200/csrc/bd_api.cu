@@ -11,6 +11,7 @@
 #include "attn_simt.cuh"
 #include "attn_tc.cuh"
 #include "kv_append.cuh"
+#include "lmhead.cuh"
 #include "unmask.cuh"
 
 namespace {
@@ -287,6 +288,112 @@ bd_status bd_kv_append(void *k_prefix, void *v_prefix, int64_t prefix_rows, cons
   p.S = S;
   p.row_vecs = row_bytes / 16;
   bd::kv_append_kernel<<<B, bd::kAppendThreads, 0, reinterpret_cast<cudaStream_t>(stream)>>>(p);
+  return check_launch();
+}
+
+// LM head + unmask: the sizes the kernels take
+bd_status lmhead_sizes_ok(int rows, int V, int D) {
+  if (rows < 0 || V < 1 || D < 1) return BD_ERR_INVALID_ARG;
+  if (rows > bd::kLhMaxRows || V > (1 << 24) || D % 64 != 0 || D > 16384) return BD_ERR_UNSUPPORTED;
+  if (sm_count() > bd::kLhMaxSms) return BD_ERR_UNSUPPORTED;
+  return BD_OK;
+}
+
+size_t bd_lmhead_unmask_workspace_bytes(int rows, int V, int D) {
+  if (lmhead_sizes_ok(rows, V, D) != BD_OK) return 0;
+  const int sms = sm_count();
+  if (sms <= 0) return 0;
+  return bd::lh_ws_layout(rows, D, sms, nullptr, nullptr);
+}
+
+bd_status bd_lmhead_unmask(const void *hidden, const void *w_vocab, const uint8_t *mask,
+                           float gamma, int32_t *tokens_out, float *conf_out, uint8_t *commit_out,
+                           uint8_t *mask_out, int rows, int V, int D, int block_S,
+                           int commit_at_least_one, void *workspace, size_t workspace_bytes,
+                           bd_stream_t stream) {
+  bd_status st = lmhead_sizes_ok(rows, V, D);
+  if (st != BD_OK) return st;
+  if (block_S < 0 || block_S > bd::kLhFinalizeRows) return BD_ERR_INVALID_ARG;
+  if (commit_at_least_one && block_S < 1) return BD_ERR_INVALID_ARG;
+  if (std::isnan(gamma)) return BD_ERR_INVALID_ARG;
+  if (rows == 0) return BD_OK;
+  if (!hidden || !w_vocab || !mask || !tokens_out || !conf_out || !commit_out || !workspace)
+    return BD_ERR_INVALID_ARG;
+  if (!aligned16(hidden) || !aligned16(w_vocab) || !aligned16(workspace) ||
+      (reinterpret_cast<uintptr_t>(tokens_out) & 3u) || (reinterpret_cast<uintptr_t>(conf_out) & 3u))
+    return BD_ERR_INVALID_ARG;
+  const int G = sm_count();
+  if (G <= 0) return BD_ERR_CUDA;
+  if (workspace_bytes < bd::lh_ws_layout(rows, D, G, nullptr, nullptr)) return BD_ERR_INVALID_ARG;
+  bd::LhParams p = {};
+  p.hidden = static_cast<const __nv_bfloat16 *>(hidden);
+  p.mask = mask;
+  p.rows = rows;
+  p.V = V;
+  p.D = D;
+  p.G = G;
+  p.rows_cap = ((rows + bd::kLhTile - 1) / bd::kLhTile) * bd::kLhTile;
+  p.wait_ns = bd::kDefaultWaitNs;
+  bd::lh_ws_layout(rows, D, G, &p.ws, static_cast<char *>(workspace));
+  cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
+
+  bd::EncodeTiledFn enc = bd::encode_tiled_fn();
+  if (!enc) return BD_ERR_CUDA;
+  CUtensorMap ma, mw;
+  if (!bd::make_map_2d(enc, &ma, p.ws.a, uint64_t(D), uint64_t(p.rows_cap)) ||
+      !bd::make_map_2d(enc, &mw, w_vocab, uint64_t(D), uint64_t(V)))
+    return BD_ERR_CUDA;
+  static std::atomic<int> smem_set{-1};
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    cudaGetLastError();
+    return BD_ERR_CUDA;
+  }
+  if (smem_set.load() != dev) {
+    if (cudaFuncSetAttribute(bd::lh_gemm_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                             int(bd::kLhSmemBytes)) != cudaSuccess) {
+      cudaGetLastError();
+      return BD_ERR_CUDA;
+    }
+    smem_set.store(dev);
+  }
+  bd::lh_gather_kernel<<<std::min(rows, 2 * G), bd::kLhGatherThreads, 0, cs>>>(p);
+  st = check_launch();
+  if (st != BD_OK) return st;
+  {
+    // programmatic launch: set-up overlaps the gather kernel
+    cudaLaunchConfig_t cfg = {};
+    cfg.gridDim = dim3(G);
+    cfg.blockDim = dim3(bd::kLhThreads);
+    cfg.dynamicSmemBytes = bd::kLhSmemBytes;
+    cfg.stream = cs;
+    cudaLaunchAttribute attr[1];
+    attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+    attr[0].val.programmaticStreamSerializationAllowed = 1;
+    cfg.attrs = attr;
+    cfg.numAttrs = 1;
+    cudaLaunchKernelEx(&cfg, bd::lh_gemm_kernel, ma, mw, p);
+  }
+  st = check_launch();
+  if (st != BD_OK) return st;
+  bd::LhFinalizeParams fp = {};
+  fp.mask = mask;
+  fp.gamma = gamma;
+  fp.tokens_out = tokens_out;
+  fp.conf_out = conf_out;
+  fp.commit_out = commit_out;
+  fp.mask_out = mask_out;
+  fp.rows = rows;
+  fp.G = G;
+  fp.rows_cap = p.rows_cap;
+  fp.block_S = block_S;
+  fp.fallback = commit_at_least_one ? 1 : 0;
+  // small CTAs (16 rows, or whole fallback blocks) so that the rows' record
+  // merges run on many SMs at once
+  fp.rows_per_cta = (block_S > 0) ? std::max(1, 16 / block_S) * block_S : 16;
+  fp.ws = p.ws;
+  const int grid = (rows + fp.rows_per_cta - 1) / fp.rows_per_cta;
+  launch_pdl(bd::lh_finalize_kernel, dim3(grid), dim3(bd::kLhFinalizeThreads), 0, cs, fp);
   return check_launch();
 }
 

@@ -1,0 +1,452 @@
+// LM head fused with confidence unmasking. The step right before Algorithm 2
+// ("Technical summary: Nemotron-TwoTower", Training and conditioning >
+// Sampling): every masked position's logits are the vocabulary projection of
+// its final hidden state, l[r, v] = sum_k hidden[r, k] * W[v, k], and
+// Algorithm 2 needs only their maximum, argmax and sum of exponentials. Here
+// the projection runs on the tensor cores and each 128 x 128 logit tile is
+// folded into per-row running (max, argmax, sum) straight out of TMEM, so the
+// [rows, V] logits never reach memory.
+//
+// Three kernels:
+//  * lh_gather_kernel - ranks of the masked rows (block scan of the mask in
+//    every CTA) and a copy of their hidden states into a dense bf16 tile
+//    [rows_cap, D] of the workspace, masked rank rho at row rho.
+//  * lh_gemm_kernel - one persistent CTA per SM over the items (n tile of
+//    128 tokens, m tile of 128 masked rows), ordered n-major so that the m
+//    tiles of one n tile run back to back and its 1 MB of W is read from HBM
+//    once. Warp 0 streams 64-wide K chunks of the A and W tiles by TMA
+//    (128-byte swizzle) through a 6-stage ring; warp 1 issues
+//    tcgen05.mma 128 x 128 x 16 into one of two TMEM accumulators; warps 2-9
+//    (two per TMEM lane quadrant, each half of the 128 columns) read the
+//    finished accumulator and fold it into the row's running record with the
+//    numerics of the unmask kernels (fp32 exponentials, fp64 sums, exact
+//    rescale, lowest index on ties) while the MMA fills the other buffer.
+//    Each thread keeps one record per m tile and writes them at the end.
+//  * lh_finalize_kernel - per masked row, merges the 2 * G records (one warp
+//    per row, every record load issued before the first merge; CTAs of 16
+//    rows, or of one fallback block), confidence = 1 / sum, commit = conf >
+//    gamma in fp64, the optional per-block fallback, and the outputs.
+#pragma once
+
+#include "attn_tc.cuh"
+#include "unmask.cuh"
+
+namespace bd {
+
+constexpr int kLhThreads = 320;
+constexpr int kLhStages = 6;
+constexpr int kLhTile = 128;       // rows of an m tile = tokens of an n tile
+constexpr int kLhChunk = 64;       // K elements per stage (128 bytes of bf16)
+constexpr uint32_t kLhPanel = 128 * 128;          // 128 rows x 128 B
+constexpr uint32_t kLhStageBytes = 2 * kLhPanel;  // A panel + W panel
+constexpr int kLhMaxRows = 4096;
+constexpr int kLhMaxMTiles = kLhMaxRows / kLhTile;
+constexpr uint32_t kLhTmemCols = 256;             // two 128-column accumulators
+constexpr int kLhGatherThreads = 256;
+constexpr int kLhFinalizeRows = 256;     // rows per finalize CTA at most
+constexpr int kLhFinalizeThreads = 256;
+constexpr int kLhMaxSms = 256;           // records per row = 2 * G <= 2 * kLhMaxSms
+constexpr int kLhRecPerLane = 2 * kLhMaxSms / 32;
+
+constexpr uint32_t kLhSmBar = kLhStages * kLhStageBytes;
+constexpr int kLhNumBars = 2 * kLhStages + 5;
+constexpr uint32_t kLhSmTmemSlot = kLhSmBar + 8 * kLhNumBars;
+constexpr uint32_t kLhSmAbort = kLhSmTmemSlot + 8;
+constexpr size_t kLhSmemBytes = kLhSmAbort + 8 + 1024;  // + alignment slack
+
+struct LhWs {
+  int *n_masked;         // [1]
+  int *rank;             // [rows]      rank among masked rows, -1 if unmasked
+  __nv_bfloat16 *a;      // [rows_cap, D] hidden states of the masked rows, by rank
+  UnmaskPart *rec;       // [rows_cap][G][2] per-row records of each CTA and column half
+};
+
+__host__ __device__ inline size_t lh_ws_layout(int rows, int D, int G, LhWs *ws, char *base) {
+  const size_t rows_cap = size_t((rows + kLhTile - 1) / kLhTile) * kLhTile;
+  size_t off = 0;
+  if (ws) ws->n_masked = reinterpret_cast<int *>(base + off);
+  off = align256(off + sizeof(int));
+  if (ws) ws->rank = reinterpret_cast<int *>(base + off);
+  off = align256(off + sizeof(int) * size_t(rows));
+  if (ws) ws->a = reinterpret_cast<__nv_bfloat16 *>(base + off);
+  off = align256(off + sizeof(__nv_bfloat16) * rows_cap * size_t(D));
+  if (ws) ws->rec = reinterpret_cast<UnmaskPart *>(base + off);
+  off = align256(off + sizeof(UnmaskPart) * size_t(G) * 2 * rows_cap);
+  return off;
+}
+
+struct LhParams {
+  const __nv_bfloat16 *hidden;
+  const uint8_t *mask;
+  int rows, V, D, G, rows_cap;
+  LhWs ws;
+  uint64_t wait_ns;
+};
+
+// 2-D tiled TMA load global -> shared memory, completion counted in bytes on
+// an mbarrier. No multicast.
+__device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap *tm, uint32_t bar,
+                                            int x, int y) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cluster.global.tile.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4}], [%2];"
+      :
+      : "r"(dst), "l"(reinterpret_cast<uint64_t>(tm)), "r"(bar), "r"(x), "r"(y)
+      : "memory");
+}
+
+// ---------------------------------------------------------------------------
+// gather: ranks of the masked rows and their hidden states, densely by rank
+// ---------------------------------------------------------------------------
+__global__ void __launch_bounds__(kLhGatherThreads) lh_gather_kernel(LhParams p) {
+  __shared__ int s_row[kLhMaxRows];  // row of masked rank rho
+  __shared__ int s_warp[32];
+  __shared__ int s_total;
+  const int tid = threadIdx.x;
+  pdl_launch_dependents();
+  const int chunk = (p.rows + kLhGatherThreads - 1) / kLhGatherThreads;
+  const int r_lo = min(p.rows, tid * chunk), r_hi = min(p.rows, r_lo + chunk);
+  int cnt = 0;
+  for (int r = r_lo; r < r_hi; ++r) cnt += (p.mask[r] != 0);
+  int total;
+  int rk = block_excl_scan(cnt, s_warp, &total);
+  for (int r = r_lo; r < r_hi; ++r) {
+    const bool mk = p.mask[r] != 0;
+    if (blockIdx.x == 0) p.ws.rank[r] = mk ? rk : -1;
+    if (mk) s_row[rk++] = r;
+  }
+  if (tid == 0) {
+    s_total = total;
+    if (blockIdx.x == 0) *p.ws.n_masked = total;
+  }
+  __syncthreads();
+  const int n = s_total;
+  const int vec = p.D / 8;  // 16-byte vectors per row
+  for (int rho = blockIdx.x; rho < n; rho += gridDim.x) {
+    const int4 *src = reinterpret_cast<const int4 *>(p.hidden + int64_t(s_row[rho]) * p.D);
+    int4 *dst = reinterpret_cast<int4 *>(p.ws.a + int64_t(rho) * p.D);
+    for (int i = tid; i < vec; i += kLhGatherThreads) dst[i] = __ldcs(src + i);
+  }
+}
+
+// ---------------------------------------------------------------------------
+// projection + fold
+// ---------------------------------------------------------------------------
+struct LhBars {
+  uint32_t full, empty, acc_full, acc_empty, done;
+  __device__ LhBars(uint32_t base) {
+    full = base;
+    empty = base + 8 * kLhStages;
+    acc_full = base + 16 * kLhStages;   // [2]
+    acc_empty = acc_full + 16;          // [2]
+    done = acc_empty + 16;
+  }
+};
+
+__global__ void __launch_bounds__(kLhThreads, 1)
+    lh_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_w,
+                   const LhParams p) {
+  extern __shared__ uint8_t smem_raw[];
+  const uint32_t raw = smem_u32(smem_raw);
+  const uint32_t sbase = (raw + 1023u) & ~1023u;
+  uint8_t *smem = smem_raw + (sbase - raw);
+  const LhBars bars(sbase + kLhSmBar);
+  uint32_t *tmem_slot = reinterpret_cast<uint32_t *>(smem + kLhSmTmemSlot);
+  volatile int *abort_flag = reinterpret_cast<volatile int *>(smem + kLhSmAbort);
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const int cta = blockIdx.x;
+
+  if (tid == 0) {
+    for (int i = 0; i < kLhStages; ++i) {
+      bar_init(bars.full + 8 * i, 1);
+      bar_init(bars.empty + 8 * i, 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      bar_init(bars.acc_full + 8 * i, 1);
+      bar_init(bars.acc_empty + 8 * i, 8);
+    }
+    bar_init(bars.done, 1);
+    *abort_flag = 0;
+    fence_barrier_init();
+    prefetch_tmap(&tm_a);
+    prefetch_tmap(&tm_w);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, kLhTmemCols);
+    tmem_relinquish();
+  }
+  // the set-up above overlaps the gather kernel; its results are read after it
+  pdl_wait_previous();
+  pdl_launch_dependents();
+  const int n_masked = *p.ws.n_masked;
+  const int n_mt = (n_masked + kLhTile - 1) / kLhTile;
+  const int n_nt = (p.V + kLhTile - 1) / kLhTile;
+  const int64_t W = int64_t(n_mt) * n_nt;
+  const int64_t e0 = W ? part_start(cta, W, p.G) : 0, e1 = W ? part_start(cta + 1, W, p.G) : 0;
+  const int nk = p.D / kLhChunk;
+  // every CTA walks the K chunks from its own starting chunk, so that the 148
+  // CTAs (all on the same m tile) do not read the same hidden-state chunk out
+  // of L2 at the same moment; each logit is still the sum over all chunks
+  const int k_rot = int((int64_t(cta) * 7) % nk);
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+  const uint64_t mp = p.wait_ns;
+
+  if (e1 <= e0) {
+    // nothing to project in this CTA's range (its records are still written)
+  } else if (warp == 0) {
+    if (lane == 0) {
+      uint32_t t = 0;
+      bool ok = true;
+      for (int64_t it = e0; ok && it < e1; ++it) {
+        const int nt = int(it / n_mt), mt = int(it % n_mt);
+        for (int kc = 0; kc < nk; ++kc, ++t) {
+          const uint32_t st = t % kLhStages;
+          if (t >= kLhStages &&
+              !tc_wait(bars.empty + 8 * st, ((t / kLhStages) - 1) & 1, mp, abort_flag)) {
+            ok = false;
+            break;
+          }
+          const uint32_t dst = sbase + st * kLhStageBytes;
+          bar_expect_tx(bars.full + 8 * st, kLhStageBytes);
+          const int kx = ((kc + k_rot) % nk) * kLhChunk;
+          tma_load_2d(dst, &tm_a, bars.full + 8 * st, kx, mt * kLhTile);
+          tma_load_2d(dst + kLhPanel, &tm_w, bars.full + 8 * st, kx, nt * kLhTile);
+        }
+      }
+      if (!ok) {
+        // the newest load of each stage must land before the CTA may exit
+        for (uint32_t k = 0; k < kLhStages && k < t; ++k) {
+          const uint32_t tl = t - 1 - k;
+          tc_wait(bars.full + 8 * (tl % kLhStages), (tl / kLhStages) & 1, mp, abort_flag);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    if (lane == 0) {
+      const uint32_t idesc = idesc_bf16(kLhTile, kLhTile, 0);
+      uint32_t t = 0;
+      bool ok = true;
+      int i = 0;
+      for (int64_t it = e0; ok && it < e1; ++it, ++i) {
+        const uint32_t ab = uint32_t(i) & 1u;
+        if (i >= 2 && !tc_wait(bars.acc_empty + 8 * ab, ((i >> 1) - 1) & 1, mp, abort_flag)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        for (int kc = 0; kc < nk; ++kc, ++t) {
+          const uint32_t st = t % kLhStages;
+          if (!tc_wait(bars.full + 8 * st, (t / kLhStages) & 1, mp, abort_flag)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t sa = sbase + st * kLhStageBytes;
+#pragma unroll
+          for (int k = 0; k < kLhChunk / 16; ++k) {
+            const uint64_t ad = sdesc_sw128(sa + uint32_t(k) * 32u, 16, 1024);
+            const uint64_t bd = sdesc_sw128(sa + kLhPanel + uint32_t(k) * 32u, 16, 1024);
+            mma_ss(tmem + ab * kLhTile, ad, bd, idesc, (kc > 0 || k > 0) ? 1u : 0u);
+          }
+          tc_commit(bars.empty + 8 * st);
+        }
+        if (!ok) break;
+        tc_commit(bars.acc_full + 8 * ab);
+      }
+      if (!ok) {
+        tc_commit(bars.done);
+        tc_wait(bars.done, 0, mp, abort_flag);
+      }
+    }
+  }
+
+  if (warp >= 2) {
+    // ------------------------------------------------------------ fold
+    const int q4 = warp & 3;         // TMEM lane quadrant = SM sub-partition
+    const int hf = (warp - 2) >> 2;  // which 64 of the 128 columns
+    const int lrow = q4 * 32 + lane;
+    float rm[kLhMaxMTiles];
+    int ri[kLhMaxMTiles];
+    double rs[kLhMaxMTiles];
+    for (int k = 0; k < n_mt; ++k) {
+      rm[k] = -INFINITY;
+      ri[k] = INT_MAX;
+      rs[k] = 0.0;
+    }
+    bool ok = true;
+    int i = 0;
+    for (int64_t it = e0; it < e1; ++it, ++i) {
+      const int nt = int(it / n_mt), mt = int(it % n_mt);
+      const uint32_t ab = uint32_t(i) & 1u;
+      ok = ok && __all_sync(0xffffffffu, tc_wait(bars.acc_full + 8 * ab, (i >> 1) & 1, mp, abort_flag));
+      tc_fence_after();
+      uint32_t r[64];
+      if (ok) tmem_ld_x64(tmem + (uint32_t(q4 * 32) << 16) + ab * kLhTile + uint32_t(hf) * 64u, r);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) bar_arrive(bars.acc_empty + 8 * ab);
+      const int rho = mt * kLhTile + lrow;
+      if (!ok || rho >= n_masked) continue;
+      const int v0 = nt * kLhTile + hf * 64;
+      const int nv = min(64, p.V - v0);  // valid columns of this half (>= 1 unless empty)
+      if (nv <= 0) continue;
+      float x[64];
+#pragma unroll
+      for (int c = 0; c < 64; ++c) x[c] = (c < nv) ? __uint_as_float(r[c]) : -INFINITY;
+      float mx[8];
+#pragma unroll
+      for (int k = 0; k < 8; ++k) mx[k] = x[k];
+#pragma unroll
+      for (int c = 8; c < 64; ++c) mx[c & 7] = fmaxf(mx[c & 7], x[c]);
+      const float bm = fmaxf(fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])),
+                             fmaxf(fmaxf(mx[4], mx[5]), fmaxf(mx[6], mx[7])));
+      float m = rm[mt];
+      double s = rs[mt];
+      if (bm > m) {
+        s = (m == -INFINITY) ? 0.0 : s * exp(double(m) - double(bm));
+        m = bm;
+        int first = 63;
+#pragma unroll
+        for (int c = 63; c >= 0; --c)
+          if (x[c] == bm) first = c;
+        ri[mt] = v0 + first;
+        rm[mt] = m;
+      }
+#pragma unroll
+      for (int c = 0; c < 64; c += 4) {
+        const float4 g = make_float4(x[c], x[c + 1], x[c + 2], x[c + 3]);
+        s += double(um_exp_sum4(g, m));
+      }
+      rs[mt] = s;
+    }
+    // one record per (CTA, column half, masked row); rows of m tiles this CTA
+    // never touched get the empty record, so the finalize merges blindly
+    for (int k = 0; k < n_mt; ++k) {
+      const int rho = k * kLhTile + lrow;
+      UnmaskPart rec;
+      rec.m = rm[k];
+      rec.idx = ri[k];
+      rec.sum = rs[k];
+      p.ws.rec[int64_t(rho) * (2 * p.G) + cta * 2 + hf] = rec;
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  if (warp == 1) tmem_dealloc(tmem, kLhTmemCols);
+}
+
+// ---------------------------------------------------------------------------
+// finalize: merge the records of each masked row, threshold, fallback
+// ---------------------------------------------------------------------------
+struct LhFinalizeParams {
+  const uint8_t *mask;
+  float gamma;
+  int32_t *tokens_out;
+  float *conf_out;
+  uint8_t *commit_out;
+  uint8_t *mask_out;
+  int rows, G, rows_cap, block_S, fallback, rows_per_cta;
+  LhWs ws;
+};
+
+__global__ void __launch_bounds__(kLhFinalizeThreads) lh_finalize_kernel(LhFinalizeParams p) {
+  __shared__ double s_conf[kLhFinalizeRows];
+  __shared__ uint8_t s_commit[kLhFinalizeRows];
+  __shared__ uint8_t s_mask[kLhFinalizeRows];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int nparts = 2 * p.G;
+  pdl_wait_previous();
+  for (int lr = warp; lr < p.rows_per_cta; lr += kLhFinalizeThreads / 32) {
+    const int r = blockIdx.x * p.rows_per_cta + lr;
+    const int rho = (r < p.rows) ? p.ws.rank[r] : -1;
+    if (lane == 0) {
+      s_mask[lr] = rho >= 0;
+      s_commit[lr] = 0;
+      s_conf[lr] = -1.0;
+    }
+    if (rho < 0) continue;
+    // all of the lane's records are requested before any is merged
+    UnmaskPart q[kLhRecPerLane];
+#pragma unroll
+    for (int j = 0; j < kLhRecPerLane; ++j) {
+      const int k = lane + 32 * j;
+      if (k < nparts) {
+        q[j] = p.ws.rec[int64_t(rho) * nparts + k];
+      } else {
+        q[j].m = -INFINITY;
+        q[j].idx = INT_MAX;
+        q[j].sum = 0.0;
+      }
+    }
+    UnmaskPart a = q[0];
+#pragma unroll
+    for (int j = 1; j < kLhRecPerLane; ++j) um_merge(a, q[j]);
+    float M = a.m;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
+    double sm = (a.m == -INFINITY) ? 0.0 : a.sum * exp(double(a.m) - double(M));
+    int ic = (a.m == M) ? a.idx : INT_MAX;
+#pragma unroll
+    for (int o = 16; o > 0; o >>= 1) {
+      sm += __shfl_xor_sync(0xffffffffu, sm, o);
+      ic = min(ic, __shfl_xor_sync(0xffffffffu, ic, o));
+    }
+    if (lane == 0) {
+      const double conf = 1.0 / sm;
+      s_conf[lr] = conf;
+      s_commit[lr] = conf > double(p.gamma);
+      p.tokens_out[r] = ic;
+      p.conf_out[r] = float(conf);
+    }
+  }
+  __syncthreads();
+  if (p.fallback) {
+    for (int lr = threadIdx.x * p.block_S; lr < p.rows_per_cta; lr += blockDim.x * p.block_S) {
+      const int r = blockIdx.x * p.rows_per_cta + lr;
+      if (r >= p.rows) break;
+      const int n = min(p.block_S, p.rows - r);
+      bool any_masked = false, any_commit = false;
+      int best = -1;
+      double bc = -1.0;
+      for (int k = 0; k < n; ++k) {
+        any_masked |= s_mask[lr + k] != 0;
+        any_commit |= s_commit[lr + k] != 0;
+        if (s_mask[lr + k] && s_conf[lr + k] > bc) {
+          bc = s_conf[lr + k];
+          best = lr + k;
+        }
+      }
+      if (any_masked && !any_commit && best >= 0) s_commit[best] = 1;
+    }
+    __syncthreads();
+  }
+  for (int lr = threadIdx.x; lr < p.rows_per_cta; lr += blockDim.x) {
+    const int r = blockIdx.x * p.rows_per_cta + lr;
+    if (r >= p.rows) break;
+    p.commit_out[r] = s_commit[lr];
+    if (p.mask_out) p.mask_out[r] = (s_mask[lr] && !s_commit[lr]) ? 1 : 0;
+  }
+}
+
+// ---------------------------------------------------------------------------
+// host side
+// ---------------------------------------------------------------------------
+// bf16 matrix [rows][D] as a 2-D map (x = k, y = row), boxes of 64 x 128
+// elements, 128-byte swizzled; rows past the end read as zero.
+inline bool make_map_2d(EncodeTiledFn enc, CUtensorMap *m, const void *base, uint64_t D,
+                        uint64_t rows) {
+  const cuuint64_t dims[2] = {D, rows};
+  const cuuint64_t strides[1] = {D * 2};
+  const cuuint32_t box[2] = {uint32_t(kLhChunk), uint32_t(kLhTile)};
+  const cuuint32_t es[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void *>(base), dims, strides, box,
+             es, CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B,
+             CU_TENSOR_MAP_L2_PROMOTION_L2_256B, CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+}  // namespace bd

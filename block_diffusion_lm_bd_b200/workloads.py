@@ -81,6 +81,12 @@ WORKLOADS = {
                 gamma=0.9, dtype=torch.bfloat16, qkv_std=1 / math.sqrt(2),
                 logit_std=math.sqrt(2), spike_max=16.0, prefix_len=8192, masked="all",
                 steps=16, commit_at_least_one=True),
+    # LM head fused with unmasking at the decode step: the 128 masked rows of
+    # the decode-step workload, hidden size D, its vocabulary and logit law
+    5: Workload(5, "LM head + unmask, decode step", B=8, H_q=32, H_kv=8, d=128, S=16,
+                V=131072, gamma=0.9, dtype=torch.bfloat16, qkv_std=1 / math.sqrt(2),
+                logit_std=math.sqrt(2), spike_max=16.0, prefix_len=4096, masked="all",
+                extra={"D": 4096}),
 }
 
 
@@ -146,6 +152,28 @@ def attention_inputs(w: Workload, device="cpu", step=0, lens=None, pad_rows=0,
         out["prefix_offset_host"] = offset.clone()
         out["total_rows"] = max(R, 1)
     return out
+
+
+def lmhead_inputs(w: Workload, device="cpu", step=0, rows=None, D=None, V=None):
+    """Hidden states bf16 [rows, D] ~ N(0, 1) and an LM head bf16 [V, D] whose
+    logits follow the unmask workloads' law: W ~ N(0, logit_std^2 / D) gives
+    logits ~ N(0, logit_std^2), and every row r gets one spike U(0, spike_max)
+    at a uniformly drawn token t_r by adding (s_r / |h_r|^2) h_r to W[t_r]
+    (rows drawing the same token share its row)."""
+    rows = w.B * w.S if rows is None else rows
+    D = w.extra.get("D", 4096) if D is None else D
+    V = w.V if V is None else V
+    gen = _dev_gen(device, w.seed(step) + 1100)
+    h = torch.randn((rows, D), generator=gen, device=device, dtype=torch.float32).to(torch.bfloat16)
+    W = torch.randn((V, D), generator=gen, device=device, dtype=torch.float32)
+    W.mul_(w.logit_std / math.sqrt(D))
+    cg = _cpu_gen(w.seed(step) + 1300)
+    pos = torch.randint(0, V, (rows,), generator=cg)
+    amp = torch.rand(rows, generator=cg, dtype=torch.float32) * w.spike_max
+    hf = h.float()
+    coef = (amp.to(device) / (hf * hf).sum(1)).unsqueeze(1)
+    W.index_add_(0, pos.to(device), coef * hf)
+    return h, W.to(torch.bfloat16)
 
 
 def initial_mask(w: Workload, rows=None, seed=None):

@@ -184,6 +184,52 @@ bd_status bd_unmask_noalloc(const float *logits, const uint8_t *mask, float gamm
                             int commit_at_least_one, bd_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
+/* LM head fused with confidence unmasking                                  */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * Workspace bytes bd_lmhead_unmask needs on the CURRENT device (depends on
+ * its SM count). Returns 0 for unsupported sizes or when no CUDA device is
+ * usable. No initialisation is needed.
+ */
+size_t bd_lmhead_unmask_workspace_bytes(int rows, int V, int D);
+
+/*
+ * Confidence unmasking of `rows` positions whose logits are the vocabulary
+ * projection of their final hidden states, computed and reduced on the fly so
+ * that the [rows, V] logits are never stored ("Technical summary:
+ * Nemotron-TwoTower", Training and conditioning > Sampling, Algorithm 2: all
+ * masked positions are predicted in parallel and the confident ones commit;
+ * the prediction is the LM head applied to the denoiser's output).
+ *
+ * For every row r with mask[r] != 0:
+ *     l[r, v]       = sum_k hidden[r, k] * w_vocab[v, k]   (bf16 inputs, products
+ *                     accumulated in float32 on the tensor cores)
+ * and then exactly what bd_unmask does with l: tokens_out[r] = argmax (lowest
+ * id on ties), conf_out[r] = 1 / sum_v exp(l[r, v] - max) (exponentials in
+ * float32, sums in float64), commit_out[r] = conf > gamma (strict, float64),
+ * the optional per-block fallback, mask_out. Rows with mask[r] == 0: their
+ * hidden state is not read, tokens_out / conf_out are left untouched,
+ * commit_out = 0. There is no bias, softcap or temperature.
+ *
+ * Arguments (all device pointers):
+ *   hidden     bf16 [rows, D]   final hidden states
+ *   w_vocab    bf16 [V, D]      LM head, one row per token
+ *   mask, gamma, tokens_out, conf_out, commit_out, mask_out, block_S,
+ *   commit_at_least_one         as for bd_unmask
+ *   workspace  >= bd_lmhead_unmask_workspace_bytes(rows, V, D) bytes
+ * Supported: rows <= 4096, 1 <= V <= 2^24, D a multiple of 64 and <= 16384,
+ * 0 <= block_S <= 256. Otherwise BD_ERR_UNSUPPORTED / BD_ERR_INVALID_ARG,
+ * and nothing is launched. Launches three kernels; every wait inside is
+ * bounded (BD_ERR_TIMEOUT in the device status).
+ */
+bd_status bd_lmhead_unmask(const void *hidden, const void *w_vocab, const uint8_t *mask,
+                           float gamma, int32_t *tokens_out, float *conf_out, uint8_t *commit_out,
+                           uint8_t *mask_out, int rows, int V, int D, int block_S,
+                           int commit_at_least_one, void *workspace, size_t workspace_bytes,
+                           bd_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
 /* Committing a finished block into the prefix cache                        */
 /* ------------------------------------------------------------------------ */
 

@@ -33,7 +33,7 @@ def test_header_declares_the_boundary():
     names = declared_functions()
     for required in ("bd_attn_step", "bd_attn_workspace_bytes", "bd_unmask",
                      "bd_unmask_workspace_bytes", "bd_get_device_status", "bd_status_string",
-                     "bd_kv_append"):
+                     "bd_kv_append", "bd_lmhead_unmask", "bd_lmhead_unmask_workspace_bytes"):
         assert required in names
 
 
@@ -182,3 +182,39 @@ def test_kv_append_host_validation(lib, kw, code):
 
 def test_kv_append_empty_batch_is_a_no_op(lib):
     assert _append(lib, B=0) == 0
+
+
+def _lmhead(lib, **kw):
+    a = dict(h=16, w=16, mk=16, gamma=0.9, tok=16, conf=16, com=16, mo=0, rows=4, V=8, D=64, bs=0,
+             fb=0, ws=16, wsb=1 << 30, st=0)
+    a.update(kw)
+    vp = lambda x: ctypes.c_void_p(x) if x else None
+    return lib.bd_lmhead_unmask(vp(a["h"]), vp(a["w"]), vp(a["mk"]), a["gamma"], vp(a["tok"]),
+                                vp(a["conf"]), vp(a["com"]), vp(a["mo"]), a["rows"], a["V"],
+                                a["D"], a["bs"], a["fb"], vp(a["ws"]), a["wsb"], vp(a["st"]))
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(rows=-1), INVALID),
+    (dict(rows=5000), UNSUPPORTED),
+    (dict(V=0), INVALID),
+    (dict(V=(1 << 24) + 1), UNSUPPORTED),
+    (dict(D=96), UNSUPPORTED),
+    (dict(D=32768), UNSUPPORTED),
+    (dict(bs=-1), INVALID),
+    (dict(bs=300), INVALID),
+    (dict(fb=1, bs=0), INVALID),
+    (dict(gamma=float("nan")), INVALID),
+    (dict(h=0), INVALID),
+    (dict(w=0), INVALID),
+    (dict(mk=0), INVALID),
+    (dict(ws=0), INVALID),
+    (dict(h=24), INVALID),                        # misaligned
+    (dict(tok=18), INVALID),
+])
+def test_lmhead_host_validation(lib, kw, code):
+    assert _lmhead(lib, **kw) == code
+
+
+def test_lmhead_zero_rows_is_a_no_op(lib):
+    assert _lmhead(lib, rows=0) == 0

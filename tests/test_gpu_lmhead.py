@@ -1,0 +1,143 @@
+"""GPU parity of bd_lmhead_unmask (LM head fused with confidence unmasking)
+against the float64 oracle.
+
+The GPU accumulates the bf16 products in float32 on the tensor cores, the
+oracle in float64, so a logit may differ by at most
+    tau = 2^-22 * (D / 16 + 16) * sum_k |h_k| |w_vk|
+(a float32 rounding of at most a few ulps for each of the D/16 accumulating
+MMA steps and inside each step, on partial sums bounded by the sum of absolute
+products). Hence: the token must equal the oracle's argmax wherever the exact
+top-two gap exceeds 2 tau; conf must agree within conf * (exp(2 tau) - 1) plus
+the 1e-6 of the unmask path; commit must agree wherever |conf - gamma| exceeds
+that tolerance. Rows inside those windows are counted and must stay rare.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from block_diffusion_lm_bd_b200 import api, workloads
+from oracle.lmhead import lmhead_logits
+from oracle.unmask import confidence_unmask
+
+pytestmark = pytest.mark.gpu
+DEV = torch.device("cuda", 0)
+W5 = workloads.WORKLOADS[5]
+
+
+def _tau(h64, W64, D):
+    return 2.0 ** -22 * (D / 16 + 16) * (np.abs(h64) @ np.abs(W64).T).max(axis=1)
+
+
+def _reference(h, W, mask, gamma, block_S=0, fallback=False, rows_sel=None, chunk=4096):
+    """Oracle logits for the selected rows (all masked rows by default), the
+    head taken in vocabulary chunks so that float64 copies stay small."""
+    m = mask.cpu().numpy().astype(bool)
+    sel = np.flatnonzero(m) if rows_sel is None else np.asarray(rows_sel)
+    V, D = W.shape
+    hs = h[torch.as_tensor(sel, device=h.device)].double().cpu().numpy()
+    logits = np.empty((sel.size, V))
+    tau = np.zeros(sel.size)
+    for v0 in range(0, V, chunk):
+        Wc = W[v0:v0 + chunk].double().cpu().numpy()
+        logits[:, v0:v0 + chunk] = lmhead_logits(hs, Wc)
+        tau = np.maximum(tau, _tau(hs, Wc, D))
+    return sel, logits, tau
+
+
+def _check(h, W, mask, gamma, block_S=0, fallback=False, workspace=None, rows_sel=None):
+    res = api.lmhead_unmask(h, W, mask, gamma, block_S=block_S, commit_at_least_one=fallback,
+                            workspace=workspace)
+    torch.cuda.synchronize()
+    assert api.get_device_status() == 0
+    sel, logits, tau = _reference(h, W, mask, gamma, block_S, fallback, rows_sel)
+    tok = res["tokens"].cpu().numpy()[sel]
+    conf = res["conf"].cpu().numpy().astype(np.float64)[sel]
+    srt = np.sort(logits, axis=1)
+    gap = srt[:, -1] - srt[:, -2] if logits.shape[1] > 1 else np.full(sel.size, np.inf)
+    ref = confidence_unmask(logits, np.ones(sel.size), gamma)
+    ok_tok = gap > 2 * tau
+    assert (tok[ok_tok] == ref["tokens"][ok_tok]).all()
+    ctol = ref["conf"] * np.expm1(2 * tau) + 1e-6
+    assert (np.abs(conf - ref["conf"]) <= ctol).all(), float(np.max(np.abs(conf - ref["conf"]) - ctol))
+    excluded = int((~ok_tok).sum())
+    if rows_sel is None and not fallback:
+        com = res["commit"].cpu().numpy().astype(bool)
+        m = mask.cpu().numpy().astype(bool)
+        assert not com[~m].any()
+        decided = np.abs(ref["conf"] - np.float64(np.float32(gamma))) > ctol
+        assert (com[sel][decided] == ref["commit"][decided]).all()
+    return res, excluded, sel.size, float(tau.max())
+
+
+@pytest.mark.parametrize("rows,D,V,frac,seed", [
+    (100, 256, 4096 + 37, 0.5, 0),     # ragged vocabulary tail, half masked
+    (129, 512, 1000, 1.0, 1),          # two m tiles, the second with one row
+    (1, 64, 1, 1.0, 2),                # one row, one token, one K chunk
+    (300, 128, 20000, 0.7, 3),         # three m tiles
+    (4096, 64, 512, 1.0, 4),           # the most rows one call takes (32 m tiles)
+])
+def test_small_cases_match_oracle(rows, D, V, frac, seed):
+    h, W = workloads.lmhead_inputs(W5.with_(V=V), device=DEV, step=seed, rows=rows, D=D, V=V)
+    g = torch.Generator().manual_seed(seed)
+    mask = (torch.rand(rows, generator=g) < frac).to(torch.uint8)
+    if frac == 1.0:
+        mask[:] = 1
+    _, excl, n, tau = _check(h, W, mask.to(DEV), W5.gamma)
+    assert excl <= max(1, n // 10), (excl, n, tau)
+
+
+def test_fallback_and_mask_out():
+    rows, D, V = 64, 256, 3000
+    h, W = workloads.lmhead_inputs(W5, device=DEV, step=7, rows=rows, D=D, V=V)
+    mask = torch.ones(rows, dtype=torch.uint8, device=DEV)
+    mask[::3] = 0
+    mask_out = torch.empty(rows, dtype=torch.uint8, device=DEV)
+    res = api.lmhead_unmask(h, W, mask, 0.999, block_S=16, commit_at_least_one=True,
+                            mask_out=mask_out)
+    torch.cuda.synchronize()
+    com = res["commit"].cpu().numpy().astype(bool)
+    m = mask.cpu().numpy().astype(bool)
+    conf = res["conf"].cpu().numpy()
+    for b in range(rows // 16):
+        sl = slice(16 * b, 16 * b + 16)
+        assert com[sl].sum() >= 1
+        # the fallback commits the masked row of highest confidence
+        if not (conf[sl][m[sl]] > np.float32(0.999)).any():
+            best = np.flatnonzero(m[sl])[np.argmax(conf[sl][m[sl]])]
+            assert com[sl].tolist() == [k == best for k in range(16)]
+    assert (mask_out.cpu().numpy().astype(bool) == (m & ~com)).all()
+    assert not com[~m].any()
+
+
+def test_unmasked_rows_untouched_and_nothing_commits():
+    h, W = workloads.lmhead_inputs(W5, device=DEV, step=8, rows=40, D=128, V=777)
+    mask = torch.zeros(40, dtype=torch.uint8, device=DEV)
+    tok = torch.full((40,), -7, dtype=torch.int32, device=DEV)
+    res = api.lmhead_unmask(h, W, mask, 0.5, tokens_out=tok)
+    torch.cuda.synchronize()
+    assert (tok.cpu() == -7).all()
+    assert not res["commit"].cpu().bool().any()
+
+
+def test_garbage_workspace_rows_do_not_leak():
+    # rows past the masked count in the gathered tile hold whatever the
+    # workspace held (here NaN bit patterns); they must not reach any output
+    rows, D, V = 100, 256, 2048
+    h, W = workloads.lmhead_inputs(W5, device=DEV, step=9, rows=rows, D=D, V=V)
+    ws = torch.full((api.lmhead_unmask_workspace_bytes(rows, V, D),), 0xFF, dtype=torch.uint8,
+                    device=DEV)
+    mask = torch.ones(rows, dtype=torch.uint8, device=DEV)
+    res, excl, n, _ = _check(h, W, mask, W5.gamma, workspace=ws)
+    assert np.isfinite(res["conf"].cpu().numpy()).all()
+
+
+def test_full_size_decode_step_sampled_rows():
+    rows = W5.B * W5.S
+    h, W = workloads.lmhead_inputs(W5, device=DEV)
+    mask = torch.ones(rows, dtype=torch.uint8, device=DEV)
+    rng = np.random.default_rng(5)
+    sel = np.unique(np.concatenate([[0, rows - 1], rng.integers(0, rows, 10)]))
+    res, excl, n, tau = _check(h, W, mask, W5.gamma, rows_sel=sel)
+    print(f"lmhead full size: {n} sampled rows, {excl} inside the tie window, tau {tau:.2e}")
+    assert excl <= 2
