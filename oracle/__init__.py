@@ -18,6 +18,9 @@ restatement of what the denoise step computes, written from the source pages:
   denoiser reads it and never writes it.
 * "Nemotron-Labs Diffusion" (molayo1419.me), diffusion mode (FastDiffuser):
   32-token blocks filled by iterative denoising with a confidence threshold.
+* The LM head in front of Algorithm 2 (``lmhead``) and the block-local
+  bidirectional Mamba scan of the partial-bidirectionality page (``mamba``),
+  each restated in its module with the readings it takes.
 
 Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline /
 reference leg may import it. The CUDA product path
@@ -33,6 +36,8 @@ from .attention import attend, block_attention, lse_combine
 from .unmask import confidence_unmask, top2_gap
 from .loop import block_loop
 from .kv_cache import kv_append
+from .lmhead import lmhead_logits, lmhead_unmask
+from .mamba import batch_block_scan, block_scan
 
 __all__ = [
     "attend",
@@ -42,4 +47,8 @@ __all__ = [
     "top2_gap",
     "block_loop",
     "kv_append",
+    "lmhead_logits",
+    "lmhead_unmask",
+    "block_scan",
+    "batch_block_scan",
 ]

@@ -17,6 +17,7 @@ import pytest
 import test_oracle_attention as TA
 import test_oracle_kv_cache as TK
 import test_oracle_lmhead as TL
+import test_oracle_mamba as TM
 import test_oracle_unmask as TU
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -148,6 +149,25 @@ def test_lmhead_mutant_is_caught(mut, monkeypatch):
     assert _some_pin_fails(TL, patches, monkeypatch), f"no pin caught mutant {name!r}"
 
 
+MAMBA_MUTANTS = [
+    ("interleaved groups", "        g = h // hpg\n", "        g = h % G\n"),
+    ("reverse scan starts from the boundary state", "        state = np.zeros_like(h0[h])\n", "        state = h0[h].copy()\n"),
+    ("skip term dropped", " + Dskip[h] * x[t, h]", ""),
+    ("decay after the input", "state = np.exp(dt[t, h] * A[h]) * state + dt[t, h] * np.outer(x[t, h], Bm[t, g])",
+     "state = np.exp(dt[t, h] * A[h]) * (state + dt[t, h] * np.outer(x[t, h], Bm[t, g]))"),
+    ("reverse uses forward step sizes", "np.exp(dt_r[t, h] * A_r[h])", "np.exp(dt[t, h] * A_r[h])"),
+    ("reverse reads C instead of C_r", "y[t, h] += state @ C_r[t, g]", "y[t, h] += state @ Cm[t, g]"),
+]
+
+
+@pytest.mark.parametrize("mut", MAMBA_MUTANTS, ids=[m[0] for m in MAMBA_MUTANTS])
+def test_mamba_mutant_is_caught(mut, monkeypatch):
+    name, old, new = mut
+    mod = _load_mutant("oracle/mamba.py", old, new, "mut_mamba")
+    patches = {"block_scan": mod.block_scan, "batch_block_scan": mod.batch_block_scan}
+    assert _some_pin_fails(TM, patches, monkeypatch), f"no pin caught mutant {name!r}"
+
+
 def test_unmutated_copy_passes_every_pin(monkeypatch):
     """Control: the loader itself does not make pins fail."""
     mod = _load_mutant("oracle/attention.py", "import numpy as np", "import numpy as np", "same_attn")
@@ -159,3 +179,6 @@ def test_unmutated_copy_passes_every_pin(monkeypatch):
                                     "top2_gap": mod.top2_gap}, monkeypatch)
     mod = _load_mutant("oracle/kv_cache.py", "import numpy as np", "import numpy as np", "same_kv")
     assert not _some_pin_fails(TK, {"kv_append": mod.kv_append}, monkeypatch)
+    mod = _load_mutant("oracle/mamba.py", "import numpy as np", "import numpy as np", "same_mamba")
+    assert not _some_pin_fails(TM, {"block_scan": mod.block_scan,
+                                    "batch_block_scan": mod.batch_block_scan}, monkeypatch)
