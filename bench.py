@@ -24,7 +24,7 @@ d=128, prefix 4096, block S=16, V=131072, gamma=0.9), synthetic data.
 * --workload 2 / 3: ragged S=32 prefixes / one 262144-token prefix; 4: the
   block loop (up to 16 steps of B=64 blocks, then the block commit into the
   prefix cache); 5: the LM head fused with unmasking (128 rows, D=4096,
-  V=131072).
+  V=131072); 6: one Mamba-2 layer's block-local bidirectional scan (B=64).
 Under torchrun (N > 1) every rank runs an independent replica (replicas
 only: the step has no exchange); the time is the max over ranks.
 """
@@ -827,6 +827,157 @@ def run_lmhead(args):
         dist.destroy_process_group()
 
 
+# --------------------------------------------------------------------------
+# block-local bidirectional Mamba scan (workload 6)
+# --------------------------------------------------------------------------
+def mamba_bytes(inp):
+    return sum(t.numel() * t.element_size() for t in inp.values()) + inp["x"].numel() * 4
+
+
+def mamba_cpu_sample(w, seconds):
+    """The oracle on one sequence's block per unit (all heads)."""
+    from block_diffusion_lm_bd_b200 import workloads
+    from oracle.mamba import block_scan
+
+    inp = workloads.mamba_inputs(w, device="cpu", B=1)
+    args = [inp[k][0] if inp[k].dim() > 1 else inp[k] for k in workloads.MAMBA_ARGS]
+    t, n = 0.0, 0
+    while t < seconds:
+        t0 = time.perf_counter()
+        block_scan(*args)
+        t += time.perf_counter() - t0
+        n += 1
+    return n * w.S / t, n, t
+
+
+def run_mamba(args):
+    """One Mamba-2 layer's block-local bidirectional scan for B=64 sequences
+    (S=16, 64 heads x 64 channels, state 128, 8 groups): the forward scan from
+    each sequence's cached boundary state (128 MiB in all, larger than L2) and
+    the reverse scan inside the block. Two rotating input sets."""
+    from block_diffusion_lm_bd_b200 import api, build as _build, workloads
+
+    world, rank, local = dist_env()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    dist = init_dist(world, "nccl")
+    if rank == 0 and _build.needs_build():
+        _build.build()
+    barrier(dist, dev)
+    w = workloads.WORKLOADS[6]
+    sets = [workloads.mamba_inputs(w, device=dev, step=1000 * rank + s) for s in range(2)]
+    ys = [torch.empty_like(s["x"]) for s in sets]
+    stream = torch.cuda.Stream(device=dev)
+
+    def call(i):
+        inp = sets[i % 2]
+        api.mamba_block_scan(*[inp[k] for k in workloads.MAMBA_ARGS], y=ys[i % 2], stream=stream)
+
+    with torch.cuda.stream(stream):
+        for i in range(max(args.warmup, 3)):
+            call(i)
+    stream.synchronize()
+    P = min(args.steps, 200)
+    n_full, tail = divmod(args.steps, P)
+    l0 = api.launch_count()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        for i in range(P):
+            call(i)
+    launches = (api.launch_count() - l0) / P
+    g_tail = None
+    if tail:
+        g_tail = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_tail, stream=stream):
+            for i in range(tail):
+                call(i)
+    g.replay()
+    torch.cuda.synchronize(dev)
+    t0 = torch.cuda.Event(enable_timing=True)
+    t1 = torch.cuda.Event(enable_timing=True)
+    sampler = ClockSampler(dev)
+    with sampler:
+        barrier(dist, dev)
+        torch.cuda.synchronize(dev)
+        with torch.cuda.stream(stream):
+            t0.record(stream)
+            for _ in range(n_full):
+                g.replay()
+            if g_tail is not None:
+                g_tail.replay()
+            t1.record(stream)
+        torch.cuda.synchronize(dev)
+        barrier(dist, dev)
+    assert api.get_device_status(stream) == 0
+    tokens = w.B * w.S
+    value, ms = aggregate_throughput(tokens * args.steps, t0.elapsed_time(t1), dist, dev)
+    call_us = ms * 1e3 / args.steps
+
+    # e2e: the block's per-token inputs from pinned host memory, y back; the
+    # boundary states and the layer's parameters are resident
+    per_token = ("x", "dt", "B_fwd", "C_fwd", "dt_rev", "B_rev", "C_rev")
+    host = {k: sets[0][k].to("cpu").pin_memory() for k in per_token}
+    y_host = torch.empty(ys[0].shape, dtype=torch.float32).pin_memory()
+    K = min(args.steps, args.e2e_steps)
+    with torch.cuda.stream(stream):
+        barrier(dist, dev)
+        t0.record(stream)
+        for _ in range(K):
+            for k in per_token:
+                sets[0][k].copy_(host[k], non_blocking=True)
+            call(0)
+            y_host.copy_(ys[0], non_blocking=True)
+        t1.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(t0.elapsed_time(t1), dist, dev)
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        v, n, t = mamba_cpu_sample(w, args.cpu_seconds)
+        cpu = {"value": v, "unit": "block-tokens/s", "cores": cpu_threads(), "kind": "oracle",
+               "sample": f"{n} units in {t:.1f} s; one sequence's block (all heads, both "
+                         "directions) per unit, float64 NumPy loops",
+               "host_cpus": len(os.sched_getaffinity(0))}
+    if rank == 0:
+        peak, peak_kind = hbm_peak()
+        nbytes = mamba_bytes(sets[0])
+        e = w.extra
+        achieved = nbytes / (call_us * 1e3)
+        rec = {
+            "metric": "Mamba block scan block-tokens/s",
+            "value": value,
+            "unit": "block-tokens/s",
+            "n_gpus": world,
+            "steps": args.steps,
+            "warmup": args.warmup,
+            "ms_per_step": ms / args.steps,
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "f32",
+            "data": "synthetic (seeded; Mamba-2 layer inputs of the stated law)",
+            "config": {"workload": f"block-local bidirectional Mamba-2 scan: B={w.B} S={w.S} "
+                                   f"H={e['H']} P={e['P']} N={e['N']} G={e['G']}, fp32 boundary "
+                                   f"states {w.B * e['H'] * e['P'] * e['N'] * 4 >> 20} MiB "
+                                   "(> L2), two rotating input sets",
+                       "parallelism": f"replicas x{world}"},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": None, "peak_kind": peak_kind,
+                         "kernel": "mamba_scan_kernel", "algorithmic_bytes": nbytes,
+                         "avg_call_us": call_us},
+            "cpu_baseline": cpu,
+            "e2e": {"value": tokens * K * world / (e2e_ms * 1e-3), "unit": "block-tokens/s",
+                    "h2d_bytes_per_step": sum(t.numel() * 4 for t in host.values()),
+                    "d2h_bytes_per_step": y_host.numel() * 4, "steps": K,
+                    "ms_per_step": e2e_ms / K},
+            "gpu_launches": int(round(launches * args.steps)),
+            "clocks": sampler.summary(),
+        }
+        print(json.dumps(rec))
+    if dist is not None:
+        dist.destroy_process_group()
+
+
 def run_reference(args):
     world, rank, _ = dist_env()
     if rank != 0:
@@ -834,6 +985,21 @@ def run_reference(args):
     from block_diffusion_lm_bd_b200 import workloads
 
     w = workloads.WORKLOADS[args.workload]
+    if args.workload == 6:
+        v, n, t = mamba_cpu_sample(w, max(1.0, min(30.0, args.steps * 0.5)))
+        rec = {"impl": "reference", "metric": "Mamba block scan block-tokens/s", "value": v,
+               "unit": "block-tokens/s", "n_gpus": world, "steps": args.steps,
+               "warmup": args.warmup, "ms_per_step": t / max(n, 1) * 1e3,
+               "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+               "data": "synthetic (seeded)", "config": {"workload": w.name,
+                                                        "parallelism": "host cores"},
+               "cpu_baseline": {"value": v, "unit": "block-tokens/s", "cores": cpu_threads(),
+                                "kind": "oracle",
+                                "sample": f"{n} units in {t:.1f} s; one sequence's block per unit"},
+               "e2e": {"value": v, "unit": "block-tokens/s", "h2d_bytes_per_step": 0,
+                       "d2h_bytes_per_step": 0}}
+        print(json.dumps(rec))
+        return
     if args.workload == 5:
         v, n, t = lmhead_cpu_sample(w, max(1.0, min(30.0, args.steps * 0.5)))
         rec = {"impl": "reference", "metric": "LM head + unmask block-tokens/s", "value": v,
@@ -887,7 +1053,7 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=4000)
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
-    ap.add_argument("--workload", type=int, default=1, choices=[1, 2, 3, 4, 5])
+    ap.add_argument("--workload", type=int, default=1, choices=[1, 2, 3, 4, 5, 6])
     ap.add_argument("--graph-steps", type=int, default=400)
     ap.add_argument("--sets", type=int, default=4,
                     help="rotating input sets (4 keep every step's inputs out of L2)")
@@ -903,6 +1069,8 @@ def main(argv=None):
         run_loop(args)
     elif args.workload == 5:
         run_lmhead(args)
+    elif args.workload == 6:
+        run_mamba(args)
     else:
         run_gpu(args)
 

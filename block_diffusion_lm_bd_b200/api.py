@@ -60,6 +60,8 @@ def _lib():
     lib.bd_lmhead_unmask.restype = i32
     lib.bd_lmhead_unmask.argtypes = [vp, vp, vp, f32, vp, vp, vp, vp, i32, i32, i32, i32, i32, vp,
                                      sz, vp]
+    lib.bd_mamba_block_scan.restype = i32
+    lib.bd_mamba_block_scan.argtypes = [vp] * 12 + [i32] * 6 + [vp]
     lib.bd_kv_append.restype = i32
     lib.bd_kv_append.argtypes = [vp, vp, i64, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, vp]
     lib.bd_get_device_status.restype = i32
@@ -223,6 +225,36 @@ def lmhead_unmask(hidden, w_vocab, mask, gamma, block_S=0, commit_at_least_one=F
         _ptr(workspace), workspace.numel() * workspace.element_size(), _stream_ptr(stream, dev))
     _check(st, "bd_lmhead_unmask")
     return {"tokens": tokens_out, "conf": conf_out, "commit": commit_out, "mask_out": mask_out}
+
+
+def mamba_block_scan(x, dt, B_fwd, C_fwd, dt_rev, B_rev, C_rev, A_fwd, A_rev, D_skip, h0, y=None,
+                     stream=None):
+    """bd_mamba_block_scan on float32 torch tensors: x [B,S,H,P], dt / dt_rev
+    [B,S,H], B/C [B,S,G,N], A_fwd / A_rev / D_skip [H], h0 [B,H,P,N]. Returns y
+    [B,S,H,P]."""
+    Bn, S, H, P = x.shape
+    G, N = B_fwd.shape[2], B_fwd.shape[3]
+    dev = x.device
+    for t, nm in ((x, "x"), (dt, "dt"), (B_fwd, "B_fwd"), (C_fwd, "C_fwd"), (dt_rev, "dt_rev"),
+                  (B_rev, "B_rev"), (C_rev, "C_rev"), (A_fwd, "A_fwd"), (A_rev, "A_rev"),
+                  (D_skip, "D_skip"), (h0, "h0")):
+        _need(t, nm, torch.float32, dev)
+    if dt.shape != (Bn, S, H) or dt_rev.shape != dt.shape:
+        raise ValueError("dt / dt_rev must be [B, S, H]")
+    for t in (C_fwd, B_rev, C_rev):
+        if t.shape != B_fwd.shape:
+            raise ValueError("B / C tensors must all be [B, S, G, N]")
+    if h0.shape != (Bn, H, P, N):
+        raise ValueError("h0 must be [B, H, P, N]")
+    if y is None:
+        y = torch.empty_like(x)
+    _need(y, "y", torch.float32, dev)
+    st = _lib().bd_mamba_block_scan(
+        _ptr(x), _ptr(dt), _ptr(B_fwd), _ptr(C_fwd), _ptr(dt_rev), _ptr(B_rev), _ptr(C_rev),
+        _ptr(A_fwd), _ptr(A_rev), _ptr(D_skip), _ptr(h0), _ptr(y), Bn, S, H, P, N, G,
+        _stream_ptr(stream, dev))
+    _check(st, "bd_mamba_block_scan")
+    return y
 
 
 def kv_append(k_prefix, v_prefix, k_new, v_new, prefix_len, prefix_offset, prefix_capacity,

@@ -12,6 +12,7 @@
 #include "attn_tc.cuh"
 #include "kv_append.cuh"
 #include "lmhead.cuh"
+#include "mamba_scan.cuh"
 #include "unmask.cuh"
 
 namespace {
@@ -394,6 +395,58 @@ bd_status bd_lmhead_unmask(const void *hidden, const void *w_vocab, const uint8_
   fp.ws = p.ws;
   const int grid = (rows + fp.rows_per_cta - 1) / fp.rows_per_cta;
   launch_pdl(bd::lh_finalize_kernel, dim3(grid), dim3(bd::kLhFinalizeThreads), 0, cs, fp);
+  return check_launch();
+}
+
+bd_status bd_mamba_block_scan(const float *x, const float *dt, const float *B_fwd,
+                              const float *C_fwd, const float *dt_rev, const float *B_rev,
+                              const float *C_rev, const float *A_fwd, const float *A_rev,
+                              const float *D_skip, const float *h0, float *y, int B, int S, int H,
+                              int P, int N, int G, bd_stream_t stream) {
+  if (B < 0 || B > bd::kMaxBatch || S < 1 || H < 1 || G < 1 || P < 1 || N < 1)
+    return BD_ERR_INVALID_ARG;
+  if (H % G != 0) return BD_ERR_INVALID_ARG;
+  if (S > bd::kMambaMaxS || (P != 32 && P != 64 && P != 128) || (N != 32 && N != 64 && N != 128) ||
+      H > 65535)
+    return BD_ERR_UNSUPPORTED;
+  if (B == 0) return BD_OK;
+  const float *in[] = {x, dt, B_fwd, C_fwd, dt_rev, B_rev, C_rev, A_fwd, A_rev, D_skip, h0};
+  for (const float *ptr : in)
+    if (!ptr || (reinterpret_cast<uintptr_t>(ptr) & 3u)) return BD_ERR_INVALID_ARG;
+  if (!y || !aligned16(h0) || !aligned16(x) || !aligned16(B_fwd) || !aligned16(C_fwd) ||
+      !aligned16(B_rev) || !aligned16(C_rev) || (reinterpret_cast<uintptr_t>(y) & 3u))
+    return BD_ERR_INVALID_ARG;
+  bd::MambaParams p = {};
+  p.x = x;
+  p.dt = dt;
+  p.Bf = B_fwd;
+  p.Cf = C_fwd;
+  p.dt_r = dt_rev;
+  p.Br = B_rev;
+  p.Cr = C_rev;
+  p.Af = A_fwd;
+  p.Ar = A_rev;
+  p.Dskip = D_skip;
+  p.h0 = h0;
+  p.y = y;
+  p.B = B;
+  p.S = S;
+  p.H = H;
+  p.P = P;
+  p.N = N;
+  p.G = G;
+  const size_t smem = bd::mamba_smem_bytes(S, P, N);
+  if (smem > 227 * 1024) return BD_ERR_UNSUPPORTED;  // the block's inputs must fit on chip
+  void (*kern)(bd::MambaParams) = N == 32 ? bd::mamba_scan_kernel<1>
+                                  : N == 64 ? bd::mamba_scan_kernel<2>
+                                            : bd::mamba_scan_kernel<4>;
+  if (smem > 48 * 1024 &&
+      cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
+          cudaSuccess) {
+    cudaGetLastError();
+    return BD_ERR_CUDA;
+  }
+  kern<<<dim3(H, B), P * (N / 32), smem, reinterpret_cast<cudaStream_t>(stream)>>>(p);
   return check_launch();
 }
 

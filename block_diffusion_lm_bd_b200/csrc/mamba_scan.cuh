@@ -1,0 +1,213 @@
+// Block-local bidirectional Mamba scan ("Training Hybrid Block Diffusion
+// Language Models with Partial Bidirectionality", Methodology: the finished
+// prefix keeps only a forward boundary state of each Mamba layer, and the
+// reverse scan is confined to the active block, so the cached state depends on
+// the clean prefix alone). Mamba-2 recurrence, per head h (scalar decay A < 0,
+// grouped B / C, head h in group h / (H / G)):
+//   forward from the cached boundary state h0:
+//     s[t] = exp(dt[t] A) s[t-1] + dt[t] x[t] B[t]^T,  y_fwd[t] = s[t] C[t] + D x[t]
+//   reverse inside the block, from zero after its last token:
+//     r[t] = exp(dt_r[t] A_r) r[t+1] + dt_r[t] x[t] B_r[t]^T,  y_rev[t] = r[t] C_r[t]
+//   y = y_fwd + y_rev.
+// The boundary state is read, never written.
+//
+// One CTA per (head, sequence); thread (c, q) owns state row q, columns
+// 32c .. 32c+31 of both directions in registers, a warp holding 32 rows of one
+// column chunk. The block's x, dt, B, C of the head's group are staged in
+// shared memory by asynchronous copies. A step is 32 FMAs of update and 32 of
+// output per thread (B / C read as warp-wide broadcasts, four independent
+// partial sums); the state is carried scaled by the running product of decays
+// so that an update is a single FMA. Bound by fp32 FMA throughput:
+// 4 * S * P * N FMAs per head and sequence against P * N * 4 bytes of boundary
+// state (read once, streaming loads).
+#pragma once
+
+#include "bd_common.cuh"
+
+namespace bd {
+
+struct MambaParams {
+  const float *x;       // [B, S, H, P]
+  const float *dt;      // [B, S, H]
+  const float *Bf;      // [B, S, G, N]
+  const float *Cf;      // [B, S, G, N]
+  const float *dt_r;    // [B, S, H]
+  const float *Br;      // [B, S, G, N]
+  const float *Cr;      // [B, S, G, N]
+  const float *Af;      // [H]
+  const float *Ar;      // [H]
+  const float *Dskip;   // [H]
+  const float *h0;      // [B, H, P, N]
+  float *y;             // [B, S, H, P]
+  int B, S, H, P, N, G;
+};
+
+constexpr int kMambaMaxS = 64;
+
+constexpr float kMambaMinScale = 0x1p-30f;  // fold the decay product into u below this
+
+// shared floats: x, dt*x, dt_r*x [S][P]; per-chunk output partials [NC][S][P];
+// B and C of both directions [S][N]; per-step a, 1/a, a_r, 1/a_r and dt, dt_r [S]
+__host__ __device__ inline size_t mamba_smem_bytes(int S, int P, int N) {
+  const int NC = N / 32;
+  return sizeof(float) * (size_t(3 + NC) * S * P + size_t(4) * S * N + size_t(6) * S);
+}
+
+// The state is kept scaled: s[t] = pi[t] * u[t] with pi[t] the product of the
+// decays since u was last renormalised, so a step is
+//     u += (dt x / pi) b     (one FMA per column)
+//     y  = pi * (u . c)      (one FMA per column, one multiply)
+// Whenever the product would fall below kMambaMinScale the decay is folded
+// into u instead (u *= pi, pi = 1), so 1/pi never exceeds 2^30 and nothing
+// overflows; the branch depends only on (sequence, head, step), so a whole CTA
+// takes it together. Returns this thread's 32 columns of u . c.
+__device__ __forceinline__ float mamba_step(float (&u)[32], float w, const float *bv,
+                                            const float *cv) {
+  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+  // the step's 64 B / C values are all requested before the first FMA; every
+  // lane of the warp reads the same addresses (one broadcast per load)
+  float4 bb[8], cc[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    bb[k] = reinterpret_cast<const float4 *>(bv)[k];
+    cc[k] = reinterpret_cast<const float4 *>(cv)[k];
+  }
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    const float4 b4 = bb[k];
+    const float4 c4 = cc[k];
+    u[4 * k] = fmaf(w, b4.x, u[4 * k]);
+    u[4 * k + 1] = fmaf(w, b4.y, u[4 * k + 1]);
+    u[4 * k + 2] = fmaf(w, b4.z, u[4 * k + 2]);
+    u[4 * k + 3] = fmaf(w, b4.w, u[4 * k + 3]);
+    acc[0] = fmaf(u[4 * k], c4.x, acc[0]);
+    acc[1] = fmaf(u[4 * k + 1], c4.y, acc[1]);
+    acc[2] = fmaf(u[4 * k + 2], c4.z, acc[2]);
+    acc[3] = fmaf(u[4 * k + 3], c4.w, acc[3]);
+  }
+  return (acc[0] + acc[1]) + (acc[2] + acc[3]);
+}
+
+__device__ __forceinline__ void cp_async16(float *smem, const float *gmem) {
+  asm volatile("cp.async.cg.shared.global [%0], [%1], 16;" ::"r"(smem_u32(smem)), "l"(gmem)
+               : "memory");
+}
+
+// Thread (c, q) = (tid / P, tid % P): state row q, columns 32c .. 32c+31. A
+// warp covers 32 rows of one column chunk, so its B / C loads are broadcasts;
+// each thread writes its chunk's part of y[t][q] to its own partial slot and
+// the chunks are summed once at the end.
+template <int NC>
+__global__ void __launch_bounds__(512, 1) mamba_scan_kernel(MambaParams p) {
+  extern __shared__ float sm[];
+  const int h = blockIdx.x, b = blockIdx.y;
+  const int S = p.S, P = p.P, N = p.N, H = p.H, G = p.G;
+  float *sx = sm;                 // x[t]            [S][P]
+  float *sxf = sx + S * P;        // dt[t] * x[t]    [S][P]
+  float *sxr = sxf + S * P;       // dt_r[t] * x[t]  [S][P]
+  float *syp = sxr + S * P;       // partials        [NC][S][P]
+  float *sBf = syp + NC * S * P;  // [S][N] each
+  float *sCf = sBf + S * N;
+  float *sBr = sCf + S * N;
+  float *sCr = sBr + S * N;
+  float *sa = sCr + S * N;        // exp(dt A), exp(-dt A), exp(dt_r A_r), exp(-dt_r A_r), dt, dt_r
+  float *sai = sa + S;
+  float *sar = sai + S;
+  float *sari = sar + S;
+  float *sdt = sari + S;
+  float *sdtr = sdt + S;
+  const int g = h / (H / G);
+  const int tid = threadIdx.x, nth = blockDim.x;
+  const float A = p.Af[h], Arv = p.Ar[h], Dk = p.Dskip[h];
+
+  // stage the block's inputs with 16-byte asynchronous copies, all in flight at once
+  const int pv = P / 4, nv = N / 4;
+  for (int v = tid; v < S * pv; v += nth) {
+    const int t = v / pv, q4 = v % pv;
+    cp_async16(sx + t * P + 4 * q4, p.x + ((int64_t(b) * S + t) * H + h) * P + 4 * q4);
+  }
+  for (int v = tid; v < S * nv; v += nth) {
+    const int t = v / nv, n = 4 * (v % nv);
+    const int64_t o = ((int64_t(b) * S + t) * G + g) * N + n;
+    const int s = t * N + n;
+    cp_async16(sBf + s, p.Bf + o);
+    cp_async16(sCf + s, p.Cf + o);
+    cp_async16(sBr + s, p.Br + o);
+    cp_async16(sCr + s, p.Cr + o);
+  }
+  asm volatile("cp.async.commit_group;" ::: "memory");
+  for (int t = tid; t < S; t += nth) {
+    const float d = p.dt[(int64_t(b) * S + t) * H + h], dr = p.dt_r[(int64_t(b) * S + t) * H + h];
+    sdt[t] = d;
+    sdtr[t] = dr;
+    sa[t] = expf(d * A);
+    sai[t] = expf(-d * A);
+    sar[t] = expf(dr * Arv);
+    sari[t] = expf(-dr * Arv);
+  }
+  const int c = tid / P, q = tid % P;
+  float u[32];
+  {
+    const float4 *src =
+        reinterpret_cast<const float4 *>(p.h0 + ((int64_t(b) * H + h) * P + q) * N + c * 32);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      const float4 v = __ldcs(src + k);
+      u[4 * k] = v.x;
+      u[4 * k + 1] = v.y;
+      u[4 * k + 2] = v.z;
+      u[4 * k + 3] = v.w;
+    }
+  }
+  asm volatile("cp.async.wait_all;" ::: "memory");
+  __syncthreads();
+  for (int i = tid; i < S * P; i += nth) {
+    const int t = i / P;
+    sxf[i] = sdt[t] * sx[i];
+    sxr[i] = sdtr[t] * sx[i];
+  }
+  __syncthreads();
+
+  float *yp = syp + c * S * P + q;
+  // forward from the boundary state
+  float pi = 1.f, ipi = 1.f;
+  for (int t = 0; t < S; ++t) {
+    pi *= sa[t];
+    ipi *= sai[t];
+    if (pi < kMambaMinScale) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) u[i] *= pi;
+      pi = 1.f;
+      ipi = 1.f;
+    }
+    const float acc = mamba_step(u, sxf[t * P + q] * ipi, sBf + t * N + c * 32, sCf + t * N + c * 32);
+    yp[t * P] = pi * acc;
+  }
+  // reverse inside the block, from zero
+#pragma unroll
+  for (int i = 0; i < 32; ++i) u[i] = 0.f;
+  pi = 1.f;
+  ipi = 1.f;
+  for (int t = S - 1; t >= 0; --t) {
+    pi *= sar[t];
+    ipi *= sari[t];
+    if (pi < kMambaMinScale) {
+#pragma unroll
+      for (int i = 0; i < 32; ++i) u[i] *= pi;
+      pi = 1.f;
+      ipi = 1.f;
+    }
+    const float acc = mamba_step(u, sxr[t * P + q] * ipi, sBr + t * N + c * 32, sCr + t * N + c * 32);
+    yp[t * P] += pi * acc;
+  }
+  __syncthreads();
+  for (int i = tid; i < S * P; i += nth) {
+    const int t = i / P, qq = i % P;
+    float acc = Dk * sx[i];
+#pragma unroll
+    for (int k = 0; k < NC; ++k) acc += syp[k * S * P + i];
+    p.y[((int64_t(b) * S + t) * H + h) * P + qq] = acc;
+  }
+}
+
+}  // namespace bd

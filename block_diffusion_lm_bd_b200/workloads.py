@@ -87,6 +87,13 @@ WORKLOADS = {
                 V=131072, gamma=0.9, dtype=torch.bfloat16, qkv_std=1 / math.sqrt(2),
                 logit_std=math.sqrt(2), spike_max=16.0, prefix_len=4096, masked="all",
                 extra={"D": 4096}),
+    # one Mamba-2 layer's block-local bidirectional scan for the loop
+    # workload's 64 sequences (B=64, S=16): 64 heads of 64 channels, state 128,
+    # 8 B/C groups
+    6: Workload(6, "block-local bidirectional Mamba scan", B=64, H_q=32, H_kv=8, d=128, S=16,
+                V=131072, gamma=0.9, dtype=torch.float32, qkv_std=1.0,
+                logit_std=math.sqrt(2), spike_max=16.0, prefix_len=8192, masked="all",
+                extra={"H": 64, "P": 64, "N": 128, "G": 8}),
 }
 
 
@@ -174,6 +181,40 @@ def lmhead_inputs(w: Workload, device="cpu", step=0, rows=None, D=None, V=None):
     coef = (amp.to(device) / (hf * hf).sum(1)).unsqueeze(1)
     W.index_add_(0, pos.to(device), coef * hf)
     return h, W.to(torch.bfloat16)
+
+
+def mamba_inputs(w: Workload, device="cpu", step=0, B=None, S=None, H=None, P=None, N=None,
+                 G=None):
+    """Inputs of one Mamba-2 layer's block scan, float32: x, B, C ~ N(0, 1);
+    step sizes log-uniform in [0.001, 0.1] (after the softplus); decays
+    A = -U(1, 16); skip D ~ U(0.5, 1.5); boundary state h0 ~ N(0, 1)."""
+    e = w.extra
+    B = w.B if B is None else B
+    S = w.S if S is None else S
+    H = e.get("H", 64) if H is None else H
+    P = e.get("P", 64) if P is None else P
+    N = e.get("N", 128) if N is None else N
+    G = e.get("G", 8) if G is None else G
+    gen = _dev_gen(device, w.seed(step) + 1500)
+
+    def normal(*shape):
+        return torch.randn(shape, generator=gen, device=device, dtype=torch.float32)
+
+    def uniform(lo, hi, *shape):
+        return lo + (hi - lo) * torch.rand(shape, generator=gen, device=device, dtype=torch.float32)
+
+    out = {"x": normal(B, S, H, P),
+           "dt": torch.exp(uniform(math.log(1e-3), math.log(1e-1), B, S, H)),
+           "B_fwd": normal(B, S, G, N), "C_fwd": normal(B, S, G, N),
+           "dt_rev": torch.exp(uniform(math.log(1e-3), math.log(1e-1), B, S, H)),
+           "B_rev": normal(B, S, G, N), "C_rev": normal(B, S, G, N),
+           "A_fwd": -uniform(1.0, 16.0, H), "A_rev": -uniform(1.0, 16.0, H),
+           "D_skip": uniform(0.5, 1.5, H), "h0": normal(B, H, P, N)}
+    return out
+
+
+MAMBA_ARGS = ("x", "dt", "B_fwd", "C_fwd", "dt_rev", "B_rev", "C_rev", "A_fwd", "A_rev", "D_skip",
+              "h0")
 
 
 def initial_mask(w: Workload, rows=None, seed=None):

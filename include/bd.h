@@ -272,6 +272,48 @@ bd_status bd_kv_append(void *k_prefix, void *v_prefix, int64_t prefix_rows, cons
                        int H_kv, int d, bd_dtype dtype, bd_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
+/* Block-local bidirectional Mamba scan                                     */
+/* ------------------------------------------------------------------------ */
+
+/*
+ * One Mamba-2 layer's scan over the active block of B sequences, both
+ * directions ("Training Hybrid Block Diffusion Language Models with Partial
+ * Bidirectionality", Methodology: a finished prefix keeps only a forward
+ * boundary state per Mamba layer; the reverse scan is confined to the active
+ * block, so the cached state is a function of the clean prefix alone). For
+ * sequence b, head h (group g = h / (H / G)) and block position t:
+ *   forward, starting from the cached boundary state h0[b, h] (P x N):
+ *     s[t] = exp(dt[t] * A_fwd[h]) * s[t-1] + dt[t] * x[t] B_fwd[t, g]^T
+ *     y_fwd[t] = s[t] C_fwd[t, g] + D_skip[h] * x[t]
+ *   reverse, inside the block only, starting from zero after position S-1:
+ *     r[t] = exp(dt_rev[t] * A_rev[h]) * r[t+1] + dt_rev[t] * x[t] B_rev[t, g]^T
+ *     y_rev[t] = r[t] C_rev[t, g]
+ *   y[b, t, h, :] = y_fwd[t] + y_rev[t]
+ * x is shared by both directions; dt / dt_rev are the step sizes after any
+ * softplus (positive); A_fwd / A_rev are the (negative) decays.
+ *
+ * Arguments (all device pointers, float32, row-major):
+ *   x            [B, S, H, P]
+ *   dt, dt_rev   [B, S, H]
+ *   B_fwd, C_fwd, B_rev, C_rev   [B, S, G, N]
+ *   A_fwd, A_rev, D_skip         [H]
+ *   h0           [B, H, P, N]   boundary state, read only
+ * x, B_fwd, C_fwd, B_rev, C_rev and h0 must be 16-byte aligned (the kernel
+ * copies them in 16-byte pieces); the other pointers 4-byte aligned.
+ *   y            [B, S, H, P]   output (must not overlap the inputs)
+ * Supported: 1 <= S <= 64; P in {32, 64, 128}; N in {32, 64, 128};
+ * H % G == 0; B <= 4096; and the block's inputs of one head must fit in
+ * shared memory: 4 * ((3 + N/32) * S * P + 4 * S * N + 6 * S) <= 227 KiB
+ * (S = 16 fits every P and N; S = 64 fits N <= 64). Otherwise BD_ERR_UNSUPPORTED / BD_ERR_INVALID_ARG and
+ * nothing is launched. Arithmetic in float32 (expf for the decays).
+ */
+bd_status bd_mamba_block_scan(const float *x, const float *dt, const float *B_fwd,
+                              const float *C_fwd, const float *dt_rev, const float *B_rev,
+                              const float *C_rev, const float *A_fwd, const float *A_rev,
+                              const float *D_skip, const float *h0, float *y, int B, int S, int H,
+                              int P, int N, int G, bd_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
 /* Status, diagnostics                                                      */
 /* ------------------------------------------------------------------------ */
 

@@ -33,7 +33,8 @@ def test_header_declares_the_boundary():
     names = declared_functions()
     for required in ("bd_attn_step", "bd_attn_workspace_bytes", "bd_unmask",
                      "bd_unmask_workspace_bytes", "bd_get_device_status", "bd_status_string",
-                     "bd_kv_append", "bd_lmhead_unmask", "bd_lmhead_unmask_workspace_bytes"):
+                     "bd_kv_append", "bd_lmhead_unmask", "bd_lmhead_unmask_workspace_bytes",
+                     "bd_mamba_block_scan"):
         assert required in names
 
 
@@ -218,3 +219,35 @@ def test_lmhead_host_validation(lib, kw, code):
 
 def test_lmhead_zero_rows_is_a_no_op(lib):
     assert _lmhead(lib, rows=0) == 0
+
+
+def _mamba(lib, **kw):
+    a = dict(ptr=16, h0=16, y=16, B=2, S=16, H=8, P=64, N=128, G=2, st=0)
+    a.update(kw)
+    vp = lambda x: ctypes.c_void_p(x) if x else None
+    ptrs = [vp(a["ptr"])] * 10 + [vp(a["h0"]), vp(a["y"])]
+    return lib.bd_mamba_block_scan(*ptrs, a["B"], a["S"], a["H"], a["P"], a["N"], a["G"],
+                                   vp(a["st"]))
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(S=0), INVALID),
+    (dict(S=65), UNSUPPORTED),
+    (dict(P=48), UNSUPPORTED),
+    (dict(N=256), UNSUPPORTED),
+    (dict(H=6, G=4), INVALID),
+    (dict(B=-1), INVALID),
+    (dict(B=5000), INVALID),
+    (dict(ptr=0), INVALID),
+    (dict(h0=0), INVALID),
+    (dict(y=0), INVALID),
+    (dict(h0=20), INVALID),                      # h0 must be 16-byte aligned
+    (dict(ptr=18), INVALID),
+    (dict(S=64, P=64, N=128), UNSUPPORTED),       # the block's inputs exceed shared memory
+])
+def test_mamba_host_validation(lib, kw, code):
+    assert _mamba(lib, **kw) == code
+
+
+def test_mamba_empty_batch_is_a_no_op(lib):
+    assert _mamba(lib, B=0) == 0

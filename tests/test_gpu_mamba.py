@@ -1,0 +1,86 @@
+"""GPU parity of bd_mamba_block_scan against the float64 oracle.
+
+Bar: max |y_gpu - y_ref| / std(y_ref) <= 2e-4. The kernel works in float32:
+each state update and each N-term output dot product round at a relative 2^-24
+per operation, so an output carries at most about (N + 2S) * 2^-24 of the sum
+of the absolute values of its terms; with random-sign terms that sum is about
+sqrt(N) times the output's spread, which gives (128 + 128) * 6e-8 * 11 ~ 2e-4
+at the largest supported sizes.
+"""
+
+import numpy as np
+import pytest
+import torch
+
+from block_diffusion_lm_bd_b200 import api, workloads
+from oracle.mamba import batch_block_scan
+
+pytestmark = pytest.mark.gpu
+DEV = torch.device("cuda", 0)
+W6 = workloads.WORKLOADS[6]
+TOL = 2e-4
+
+
+def _run(inp):
+    y = api.mamba_block_scan(*[inp[k] for k in workloads.MAMBA_ARGS])
+    torch.cuda.synchronize()
+    assert api.get_device_status() == 0
+    return y
+
+
+def _err(y, ref):
+    return float(np.abs(y.cpu().double().numpy() - ref).max() / ref.std())
+
+
+@pytest.mark.parametrize("B,S,H,P,N,G", [
+    (2, 16, 8, 64, 128, 2),
+    (3, 1, 4, 32, 32, 4),
+    (1, 64, 2, 128, 64, 1),
+    (5, 7, 16, 32, 128, 8),
+    (2, 33, 6, 128, 128, 3),
+])
+def test_small_cases_match_oracle(B, S, H, P, N, G):
+    inp = workloads.mamba_inputs(W6, device=DEV, B=B, S=S, H=H, P=P, N=N, G=G)
+    h0 = inp["h0"].clone()
+    y = _run(inp)
+    ref = batch_block_scan(*[inp[k] for k in workloads.MAMBA_ARGS])
+    err = _err(y, ref)
+    assert err <= TOL, err
+    assert torch.equal(h0, inp["h0"]), "the boundary state must not be written"
+
+
+def test_full_size_sampled_sequences():
+    inp = workloads.mamba_inputs(W6, device=DEV)
+    y = _run(inp)
+    for b in (0, W6.B - 1, 17):
+        one = {k: (v[b:b + 1] if v.dim() > 1 else v) for k, v in inp.items()}
+        ref = batch_block_scan(*[one[k] for k in workloads.MAMBA_ARGS])
+        err = _err(y[b:b + 1], ref)
+        assert err <= TOL, (b, err)
+
+
+def test_reverse_direction_sees_only_the_block():
+    # changing the boundary state changes only the forward contribution: the
+    # difference of two outputs is exactly the decayed boundary term
+    inp = workloads.mamba_inputs(W6, device=DEV, B=2, S=8, H=4, P=32, N=64, G=2)
+    y1 = _run(inp).cpu().double().numpy()
+    inp2 = dict(inp)
+    inp2["h0"] = torch.zeros_like(inp["h0"])
+    y0 = _run(inp2).cpu().double().numpy()
+    ref1 = batch_block_scan(*[inp[k] for k in workloads.MAMBA_ARGS])
+    ref0 = batch_block_scan(*[inp2[k] for k in workloads.MAMBA_ARGS])
+    d, dref = y1 - y0, ref1 - ref0
+    assert np.abs(d - dref).max() <= TOL * ref1.std()
+
+
+def test_strong_decay_does_not_overflow_the_scaled_state():
+    # dt * |A| up to 60 per step: the decay product leaves the float32 range
+    # within two steps, so the kernel must fold it into the state
+    inp = workloads.mamba_inputs(W6, device=DEV, B=2, S=24, H=4, P=32, N=64, G=2)
+    inp["dt"] = inp["dt"] * 0 + torch.rand_like(inp["dt"]) * 4.0
+    inp["dt_rev"] = inp["dt_rev"] * 0 + torch.rand_like(inp["dt_rev"]) * 4.0
+    inp["A_fwd"] = inp["A_fwd"] * 0 - 15.0
+    y = _run(inp)
+    assert torch.isfinite(y).all()
+    ref = batch_block_scan(*[inp[k] for k in workloads.MAMBA_ARGS])
+    assert _err(y, ref) <= TOL
