@@ -942,7 +942,17 @@ def run_mamba(args):
         peak, peak_kind = hbm_peak()
         nbytes = mamba_bytes(sets[0])
         e = w.extra
-        achieved = nbytes / (call_us * 1e3)
+        # fp32 FMA peak from the unit counts and the clock: 148 SMs x 128
+        # lanes x 2 flop x max SM clock (1965 MHz), the ALU roofline of the scan
+        sm_mhz = 1965.0
+        try:
+            with open(PEAKS_FILE) as f:
+                sm_mhz = float(json.load(f).get("sm_max_mhz", sm_mhz))
+        except Exception:
+            pass
+        alu_peak = torch.cuda.get_device_properties(dev).multi_processor_count * 128 * 2 * sm_mhz * 1e6 / 1e12
+        flops = 8.0 * w.S * e["P"] * e["N"] * e["H"] * w.B  # both directions: update + output FMA
+        achieved = flops / (call_us * 1e-6) / 1e12
         rec = {
             "metric": "Mamba block scan block-tokens/s",
             "value": value,
@@ -961,10 +971,13 @@ def run_mamba(args):
                                    f"states {w.B * e['H'] * e['P'] * e['N'] * 4 >> 20} MiB "
                                    "(> L2), two rotating input sets",
                        "parallelism": f"replicas x{world}"},
-            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
-                         "frac": achieved / peak, "traffic": None, "peak_kind": peak_kind,
-                         "kernel": "mamba_scan_kernel", "algorithmic_bytes": nbytes,
-                         "avg_call_us": call_us},
+            "roofline": {"bound": "alu", "achieved": achieved, "peak": alu_peak,
+                         "unit": "TFLOP/s", "frac": achieved / alu_peak, "traffic": None,
+                         "peak_kind": "derived: SMs x 128 fp32 lanes x 2 x max SM clock",
+                         "kernel": "mamba_scan_kernel", "algorithmic_flops": flops,
+                         "avg_call_us": call_us, "hbm_bytes": nbytes,
+                         "hbm_gbs": nbytes / (call_us * 1e3), "hbm_peak": peak,
+                         "hbm_peak_kind": peak_kind},
             "cpu_baseline": cpu,
             "e2e": {"value": tokens * K * world / (e2e_ms * 1e-3), "unit": "block-tokens/s",
                     "h2d_bytes_per_step": sum(t.numel() * 4 for t in host.values()),

@@ -437,16 +437,20 @@ bd_status bd_mamba_block_scan(const float *x, const float *dt, const float *B_fw
   p.G = G;
   const size_t smem = bd::mamba_smem_bytes(S, P, N);
   if (smem > 227 * 1024) return BD_ERR_UNSUPPORTED;  // the block's inputs must fit on chip
-  void (*kern)(bd::MambaParams) = N == 32 ? bd::mamba_scan_kernel<1>
-                                  : N == 64 ? bd::mamba_scan_kernel<2>
-                                            : bd::mamba_scan_kernel<4>;
+  // two state rows per thread when that still leaves whole warps
+  const int rb = (P / 2) * (N / 32) >= 32 && P >= 64 ? 2 : 1;
+  void (*kern)(bd::MambaParams) =
+      rb == 2 ? (N == 32 ? bd::mamba_scan_kernel<1, 2>
+                         : N == 64 ? bd::mamba_scan_kernel<2, 2> : bd::mamba_scan_kernel<4, 2>)
+              : (N == 32 ? bd::mamba_scan_kernel<1, 1>
+                         : N == 64 ? bd::mamba_scan_kernel<2, 1> : bd::mamba_scan_kernel<4, 1>);
   if (smem > 48 * 1024 &&
       cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, int(smem)) !=
           cudaSuccess) {
     cudaGetLastError();
     return BD_ERR_CUDA;
   }
-  kern<<<dim3(H, B), P * (N / 32), smem, reinterpret_cast<cudaStream_t>(stream)>>>(p);
+  kern<<<dim3(H, B), (P / rb) * (N / 32), smem, reinterpret_cast<cudaStream_t>(stream)>>>(p);
   return check_launch();
 }
 

@@ -60,10 +60,15 @@ __host__ __device__ inline size_t mamba_smem_bytes(int S, int P, int N) {
 // Whenever the product would fall below kMambaMinScale the decay is folded
 // into u instead (u *= pi, pi = 1), so 1/pi never exceeds 2^30 and nothing
 // overflows; the branch depends only on (sequence, head, step), so a whole CTA
-// takes it together. Returns this thread's 32 columns of u . c.
-__device__ __forceinline__ float mamba_step(float (&u)[32], float w, const float *bv,
-                                            const float *cv) {
-  float acc[4] = {0.f, 0.f, 0.f, 0.f};
+// takes it together. A thread carries RB rows of one 32-column chunk, so each
+// of the step's B / C values it loads feeds RB updates and RB output terms.
+// acc[r] receives row r's 32-column part of u . c.
+template <int RB>
+__device__ __forceinline__ void mamba_step(float (&u)[RB][32], const float (&w)[RB],
+                                           const float *bv, const float *cv, float (&acc)[RB]) {
+  float part[RB][2];
+#pragma unroll
+  for (int r = 0; r < RB; ++r) part[r][0] = part[r][1] = 0.f;
   // the step's 64 B / C values are all requested before the first FMA; every
   // lane of the warp reads the same addresses (one broadcast per load)
   float4 bb[8], cc[8];
@@ -74,18 +79,19 @@ __device__ __forceinline__ float mamba_step(float (&u)[32], float w, const float
   }
 #pragma unroll
   for (int k = 0; k < 8; ++k) {
-    const float4 b4 = bb[k];
-    const float4 c4 = cc[k];
-    u[4 * k] = fmaf(w, b4.x, u[4 * k]);
-    u[4 * k + 1] = fmaf(w, b4.y, u[4 * k + 1]);
-    u[4 * k + 2] = fmaf(w, b4.z, u[4 * k + 2]);
-    u[4 * k + 3] = fmaf(w, b4.w, u[4 * k + 3]);
-    acc[0] = fmaf(u[4 * k], c4.x, acc[0]);
-    acc[1] = fmaf(u[4 * k + 1], c4.y, acc[1]);
-    acc[2] = fmaf(u[4 * k + 2], c4.z, acc[2]);
-    acc[3] = fmaf(u[4 * k + 3], c4.w, acc[3]);
+    const float bk[4] = {bb[k].x, bb[k].y, bb[k].z, bb[k].w};
+    const float ck[4] = {cc[k].x, cc[k].y, cc[k].z, cc[k].w};
+#pragma unroll
+    for (int r = 0; r < RB; ++r) {
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        u[r][4 * k + j] = fmaf(w[r], bk[j], u[r][4 * k + j]);
+        part[r][j & 1] = fmaf(u[r][4 * k + j], ck[j], part[r][j & 1]);
+      }
+    }
   }
-  return (acc[0] + acc[1]) + (acc[2] + acc[3]);
+#pragma unroll
+  for (int r = 0; r < RB; ++r) acc[r] = part[r][0] + part[r][1];
 }
 
 __device__ __forceinline__ void cp_async16(float *smem, const float *gmem) {
@@ -93,15 +99,17 @@ __device__ __forceinline__ void cp_async16(float *smem, const float *gmem) {
                : "memory");
 }
 
-// Thread (c, q) = (tid / P, tid % P): state row q, columns 32c .. 32c+31. A
-// warp covers 32 rows of one column chunk, so its B / C loads are broadcasts;
-// each thread writes its chunk's part of y[t][q] to its own partial slot and
-// the chunks are summed once at the end.
-template <int NC>
+// Thread (c, q) = (tid / (P/RB), tid % (P/RB)): state rows q + j * P/RB
+// (j < RB), columns 32c .. 32c+31. A warp covers 32 row slots of one column
+// chunk, so its B / C loads are broadcasts; each thread writes its chunk's
+// part of y[t][row] to its own partial slot and the chunks are summed once at
+// the end.
+template <int NC, int RB>
 __global__ void __launch_bounds__(512, 1) mamba_scan_kernel(MambaParams p) {
   extern __shared__ float sm[];
   const int h = blockIdx.x, b = blockIdx.y;
   const int S = p.S, P = p.P, N = p.N, H = p.H, G = p.G;
+  const int PR = P / RB;          // row slots per column chunk
   float *sx = sm;                 // x[t]            [S][P]
   float *sxf = sx + S * P;        // dt[t] * x[t]    [S][P]
   float *sxr = sxf + S * P;       // dt_r[t] * x[t]  [S][P]
@@ -145,18 +153,19 @@ __global__ void __launch_bounds__(512, 1) mamba_scan_kernel(MambaParams p) {
     sar[t] = expf(dr * Arv);
     sari[t] = expf(-dr * Arv);
   }
-  const int c = tid / P, q = tid % P;
-  float u[32];
-  {
-    const float4 *src =
-        reinterpret_cast<const float4 *>(p.h0 + ((int64_t(b) * H + h) * P + q) * N + c * 32);
+  const int c = tid / PR, q0 = tid % PR;
+  float u[RB][32];
+#pragma unroll
+  for (int r = 0; r < RB; ++r) {
+    const float4 *src = reinterpret_cast<const float4 *>(
+        p.h0 + ((int64_t(b) * H + h) * P + q0 + r * PR) * N + c * 32);
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
       const float4 v = __ldcs(src + k);
-      u[4 * k] = v.x;
-      u[4 * k + 1] = v.y;
-      u[4 * k + 2] = v.z;
-      u[4 * k + 3] = v.w;
+      u[r][4 * k] = v.x;
+      u[r][4 * k + 1] = v.y;
+      u[r][4 * k + 2] = v.z;
+      u[r][4 * k + 3] = v.w;
     }
   }
   asm volatile("cp.async.wait_all;" ::: "memory");
@@ -168,7 +177,8 @@ __global__ void __launch_bounds__(512, 1) mamba_scan_kernel(MambaParams p) {
   }
   __syncthreads();
 
-  float *yp = syp + c * S * P + q;
+  float *yp = syp + c * S * P + q0;
+  float w[RB], acc[RB];
   // forward from the boundary state
   float pi = 1.f, ipi = 1.f;
   for (int t = 0; t < S; ++t) {
@@ -176,16 +186,23 @@ __global__ void __launch_bounds__(512, 1) mamba_scan_kernel(MambaParams p) {
     ipi *= sai[t];
     if (pi < kMambaMinScale) {
 #pragma unroll
-      for (int i = 0; i < 32; ++i) u[i] *= pi;
+      for (int r = 0; r < RB; ++r)
+#pragma unroll
+        for (int i = 0; i < 32; ++i) u[r][i] *= pi;
       pi = 1.f;
       ipi = 1.f;
     }
-    const float acc = mamba_step(u, sxf[t * P + q] * ipi, sBf + t * N + c * 32, sCf + t * N + c * 32);
-    yp[t * P] = pi * acc;
+#pragma unroll
+    for (int r = 0; r < RB; ++r) w[r] = sxf[t * P + q0 + r * PR] * ipi;
+    mamba_step<RB>(u, w, sBf + t * N + c * 32, sCf + t * N + c * 32, acc);
+#pragma unroll
+    for (int r = 0; r < RB; ++r) yp[t * P + r * PR] = pi * acc[r];
   }
   // reverse inside the block, from zero
 #pragma unroll
-  for (int i = 0; i < 32; ++i) u[i] = 0.f;
+  for (int r = 0; r < RB; ++r)
+#pragma unroll
+    for (int i = 0; i < 32; ++i) u[r][i] = 0.f;
   pi = 1.f;
   ipi = 1.f;
   for (int t = S - 1; t >= 0; --t) {
@@ -193,20 +210,25 @@ __global__ void __launch_bounds__(512, 1) mamba_scan_kernel(MambaParams p) {
     ipi *= sari[t];
     if (pi < kMambaMinScale) {
 #pragma unroll
-      for (int i = 0; i < 32; ++i) u[i] *= pi;
+      for (int r = 0; r < RB; ++r)
+#pragma unroll
+        for (int i = 0; i < 32; ++i) u[r][i] *= pi;
       pi = 1.f;
       ipi = 1.f;
     }
-    const float acc = mamba_step(u, sxr[t * P + q] * ipi, sBr + t * N + c * 32, sCr + t * N + c * 32);
-    yp[t * P] += pi * acc;
+#pragma unroll
+    for (int r = 0; r < RB; ++r) w[r] = sxr[t * P + q0 + r * PR] * ipi;
+    mamba_step<RB>(u, w, sBr + t * N + c * 32, sCr + t * N + c * 32, acc);
+#pragma unroll
+    for (int r = 0; r < RB; ++r) yp[t * P + r * PR] += pi * acc[r];
   }
   __syncthreads();
   for (int i = tid; i < S * P; i += nth) {
     const int t = i / P, qq = i % P;
-    float acc = Dk * sx[i];
+    float v = Dk * sx[i];
 #pragma unroll
-    for (int k = 0; k < NC; ++k) acc += syp[k * S * P + i];
-    p.y[((int64_t(b) * S + t) * H + h) * P + qq] = acc;
+    for (int k = 0; k < NC; ++k) v += syp[k * S * P + i];
+    p.y[((int64_t(b) * S + t) * H + h) * P + qq] = v;
   }
 }
 
