@@ -20,7 +20,8 @@ restatement of what the denoise step computes, written from the source pages:
   32-token blocks filled by iterative denoising with a confidence threshold.
 * The LM head in front of Algorithm 2 (``lmhead``) and the block-local
   bidirectional Mamba scan of the partial-bidirectionality page (``mamba``),
-  each restated in its module with the readings it takes.
+  and self-speculative verification (``spec``: "Nemotron-Labs Diffusion",
+  self-speculation mode), each restated in its module with its readings.
 
 Only ``tests/``, ``__graft_entry__.smoke()`` and ``bench.py``'s CPU-baseline /
 reference leg may import it. The CUDA product path
@@ -38,6 +39,7 @@ from .loop import block_loop
 from .kv_cache import kv_append
 from .lmhead import lmhead_logits, lmhead_unmask
 from .mamba import batch_block_scan, block_scan
+from .spec import causal_block_attention, verify_commit
 
 __all__ = [
     "attend",
@@ -51,4 +53,6 @@ __all__ = [
     "lmhead_unmask",
     "block_scan",
     "batch_block_scan",
+    "causal_block_attention",
+    "verify_commit",
 ]

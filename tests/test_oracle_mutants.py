@@ -18,6 +18,7 @@ import test_oracle_attention as TA
 import test_oracle_kv_cache as TK
 import test_oracle_lmhead as TL
 import test_oracle_mamba as TM
+import test_oracle_spec as TS
 import test_oracle_unmask as TU
 
 ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
@@ -166,6 +167,33 @@ def test_mamba_mutant_is_caught(mut, monkeypatch):
     mod = _load_mutant("oracle/mamba.py", old, new, "mut_mamba")
     patches = {"block_scan": mod.block_scan, "batch_block_scan": mod.batch_block_scan}
     assert _some_pin_fails(TM, patches, monkeypatch), f"no pin caught mutant {name!r}"
+
+
+SPEC_MUTANTS = [
+    ("block keys not causal", "k_blk[b, :i + 1, kv]], axis=0)\n                V = np.concatenate([v_prefix[off:off + L, kv], v_blk[b, :i + 1, kv]]",
+     "k_blk[b, :, kv]], axis=0)\n                V = np.concatenate([v_prefix[off:off + L, kv], v_blk[b, :, kv]]"),
+    ("causal excludes the diagonal", "k_blk[b, :i + 1, kv]], axis=0)\n                V = np.concatenate([v_prefix[off:off + L, kv], v_blk[b, :i + 1, kv]]",
+     "k_blk[b, :max(i, 1), kv]], axis=0)\n                V = np.concatenate([v_prefix[off:off + L, kv], v_blk[b, :max(i, 1), kv]]"),
+    ("no correction token", "            commit[b * S + n] = True  # the autoregressive token at the first mismatch\n",
+     "            pass\n"),
+    ("ties to the highest id", "tokens[r] = int(np.flatnonzero(x[r] == x[r].max())[0])",
+     "tokens[r] = int(np.flatnonzero(x[r] == x[r].max())[-1])"),
+    ("accepts past a mismatch", "        commit[b * S:b * S + n] = True\n", "        commit[b * S:b * S + S] = True\n"),
+]
+
+
+@pytest.mark.parametrize("mut", SPEC_MUTANTS, ids=[m[0] for m in SPEC_MUTANTS])
+def test_spec_mutant_is_caught(mut, monkeypatch):
+    name, old, new = mut
+    src = open(os.path.join(ROOT, "oracle/spec.py")).read()
+    assert src.count(old) >= 1, old
+    spec = importlib.util.spec_from_loader("oracle._mut_spec", loader=None)
+    mod = importlib.util.module_from_spec(spec)
+    mod.__package__ = "oracle"
+    exec(compile(src.replace(old, new), "<mutant spec>", "exec"), mod.__dict__)
+    patches = {"causal_block_attention": mod.causal_block_attention,
+               "verify_commit": mod.verify_commit}
+    assert _some_pin_fails(TS, patches, monkeypatch), f"no pin caught mutant {name!r}"
 
 
 def test_unmutated_copy_passes_every_pin(monkeypatch):
