@@ -62,6 +62,13 @@ def _lib():
                                      sz, vp]
     lib.bd_mamba_block_scan.restype = i32
     lib.bd_mamba_block_scan.argtypes = [vp] * 12 + [i32] * 6 + [vp]
+    lib.bd_attn_step_ex.restype = i32
+    lib.bd_attn_step_ex.argtypes = [vp, vp, vp, i64, vp, vp, vp, vp, i32, i32, i32, i32, i32, f32,
+                                    i32, vp, vp, vp, sz, i32, vp]
+    lib.bd_spec_verify_workspace_bytes.restype = sz
+    lib.bd_spec_verify_workspace_bytes.argtypes = [i32, i32]
+    lib.bd_spec_verify.restype = i32
+    lib.bd_spec_verify.argtypes = [vp, vp, vp, vp, vp, vp, i32, i32, i32, vp, sz, vp]
     lib.bd_kv_append.restype = i32
     lib.bd_kv_append.argtypes = [vp, vp, i64, vp, vp, vp, vp, vp, vp, i32, i32, i32, i32, i32, vp]
     lib.bd_get_device_status.restype = i32
@@ -115,9 +122,13 @@ def unmask_workspace_bytes(rows, V):
     return int(_lib().bd_unmask_workspace_bytes(rows, V))
 
 
+BD_ATTN_BLOCK_CAUSAL = 1
+
+
 def attn_step(q, k_prefix, v_prefix, k_blk, v_blk, prefix_len, prefix_offset, scale=None,
-              o=None, lse=None, want_lse=True, workspace=None, stream=None):
-    """bd_attn_step on torch tensors. Returns (o float32 [B,S,H_q,d], lse or None)."""
+              o=None, lse=None, want_lse=True, workspace=None, stream=None, block_causal=False):
+    """bd_attn_step on torch tensors (bd_attn_step_ex with BD_ATTN_BLOCK_CAUSAL
+    when block_causal). Returns (o float32 [B,S,H_q,d], lse or None)."""
     B, S, H_q, d = q.shape
     H_kv = k_blk.shape[2]
     dev = q.device
@@ -144,12 +155,14 @@ def attn_step(q, k_prefix, v_prefix, k_blk, v_blk, prefix_len, prefix_offset, sc
         if nbytes == 0:
             raise BdError(1, "bd_attn_workspace_bytes")
         workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev)
-    st = _lib().bd_attn_step(
-        _ptr(q), _ptr(k_prefix), _ptr(v_prefix), int(k_prefix.shape[0]), _ptr(k_blk),
-        _ptr(v_blk), _ptr(prefix_len), _ptr(prefix_offset), B, S, H_q, H_kv, d,
-        float(scale) if scale is not None else 0.0, _DTYPES[q.dtype], _ptr(o), _ptr(lse),
-        _ptr(workspace), workspace.numel() * workspace.element_size(),
-        _stream_ptr(stream, dev))
+    args = (_ptr(q), _ptr(k_prefix), _ptr(v_prefix), int(k_prefix.shape[0]), _ptr(k_blk),
+            _ptr(v_blk), _ptr(prefix_len), _ptr(prefix_offset), B, S, H_q, H_kv, d,
+            float(scale) if scale is not None else 0.0, _DTYPES[q.dtype], _ptr(o), _ptr(lse),
+            _ptr(workspace), workspace.numel() * workspace.element_size())
+    if block_causal:
+        st = _lib().bd_attn_step_ex(*args, BD_ATTN_BLOCK_CAUSAL, _stream_ptr(stream, dev))
+    else:
+        st = _lib().bd_attn_step(*args, _stream_ptr(stream, dev))
     _check(st, "bd_attn_step")
     return o, lse
 
@@ -255,6 +268,37 @@ def mamba_block_scan(x, dt, B_fwd, C_fwd, dt_rev, B_rev, C_rev, A_fwd, A_rev, D_
         _stream_ptr(stream, dev))
     _check(st, "bd_mamba_block_scan")
     return y
+
+
+def spec_verify(logits, draft, S, tokens_out=None, conf_out=None, commit_out=None,
+                n_accept_out=None, workspace=None, stream=None):
+    """bd_spec_verify on torch tensors: logits float32 [rows, V], draft int32
+    [rows], blocks of S rows. Returns dict tokens, conf, commit, n_accept."""
+    rows, V = logits.shape
+    dev = logits.device
+    _need(logits, "logits", torch.float32, dev)
+    _need(draft, "draft", torch.int32, dev)
+    if draft.shape != (rows,) or rows % S:
+        raise ValueError("draft must be [rows] and rows a multiple of S")
+    if tokens_out is None:
+        tokens_out = torch.empty(rows, dtype=torch.int32, device=dev)
+    if conf_out is None:
+        conf_out = torch.empty(rows, dtype=torch.float32, device=dev)
+    if commit_out is None:
+        commit_out = torch.empty(rows, dtype=torch.uint8, device=dev)
+    if n_accept_out is None:
+        n_accept_out = torch.empty(rows // S, dtype=torch.int32, device=dev)
+    if workspace is None:
+        nbytes = int(_lib().bd_spec_verify_workspace_bytes(rows, V))
+        if nbytes == 0:
+            raise BdError(1, "bd_spec_verify_workspace_bytes")
+        workspace = torch.empty(nbytes, dtype=torch.uint8, device=dev)
+    st = _lib().bd_spec_verify(
+        _ptr(logits), _ptr(draft), _ptr(tokens_out), _ptr(conf_out), _ptr(commit_out),
+        _ptr(n_accept_out), rows, V, int(S), _ptr(workspace),
+        workspace.numel() * workspace.element_size(), _stream_ptr(stream, dev))
+    _check(st, "bd_spec_verify")
+    return {"tokens": tokens_out, "conf": conf_out, "commit": commit_out, "n_accept": n_accept_out}
 
 
 def kv_append(k_prefix, v_prefix, k_new, v_new, prefix_len, prefix_offset, prefix_capacity,

@@ -64,6 +64,7 @@ struct AttnParams {
   int G;
   uint64_t wait_ns;  // time limit of every barrier wait
   int q_spread;  // tensor-core kernel: Q rows spread over the TMEM lane quadrants
+  int block_causal;  // 1: block position i sees block keys 0 .. i only (verification pass)
 };
 
 __device__ __forceinline__ int attn_units(int L) { return (L + kUnitKeys - 1) / kUnitKeys + 1; }

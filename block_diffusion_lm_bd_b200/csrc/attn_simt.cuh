@@ -102,7 +102,7 @@ __global__ void __launch_bounds__(kSimtThreads, 1) attn_simt_kernel(AttnParams p
         kbase = kpg + (r0 * p.H_kv + kv) * D;
         vbase = vpg + (r0 * p.H_kv + kv) * D;
       } else {
-        cnt = p.S;
+        cnt = p.S;  // the block's own keys (causal: row m sees keys 0 .. m / g)
         kbase = kbg + (int64_t(b) * p.S * p.H_kv + kv) * D;
         vbase = vbg + (int64_t(b) * p.S * p.H_kv + kv) * D;
       }
@@ -141,7 +141,9 @@ __global__ void __launch_bounds__(kSimtThreads, 1) attn_simt_kernel(AttnParams p
 #pragma unroll
         for (int i = 0; i < 16; ++i) {
           if (i < nrw) {
-            const float x = (lane < nj) ? sc[i] * p.scale_log2 : -INFINITY;
+            const bool seen = lane < nj && !(p.block_causal && u == n - 1 &&
+                                             j0 + lane > (warp + 8 * i) / g);
+            const float x = seen ? sc[i] * p.scale_log2 : -INFINITY;
             const float mn = fmaxf(mrow[i], warp_max(x));
             const float alpha = exp2f(mrow[i] - mn);
             const float pv = exp2f(x - mn);

@@ -342,6 +342,8 @@ __global__ void __launch_bounds__(kTcThreads, 1)
       m = lq;
     }
     const bool active = p.q_spread || q4 * 32 < p.M;  // same for both warps of a quadrant
+    // keys of the block tile this row sees: all S, or 0 .. its own position
+    const int blk_valid = p.block_causal ? min(p.S, m / p.g + 1) : p.S;
     const uint32_t lrow = uint32_t(q4 * 32) << 16;
     const uint32_t col0 = uint32_t(hf) * 64u;      // score / O columns of this half
     const uint32_t bar_id = 1u + uint32_t(q4);     // named barrier of the quadrant's pair
@@ -363,7 +365,7 @@ __global__ void __launch_bounds__(kTcThreads, 1)
         ok = ok && __all_sync(0xffffffffu, tc_wait(bars.s_full + 8 * sb, (t >> 1) & 1, mp, abort_flag));
         tc_fence_after();
         const bool blk = (u == wk.sn - 1);
-        const int nvalid = blk ? p.S : min(kTcKeys, wk.sL - u * kTcKeys);
+        const int nvalid = blk ? blk_valid : min(kTcKeys, wk.sL - u * kTcKeys);
         float alpha = 1.f;
         bool resc = false;
         if (active) {

@@ -13,6 +13,7 @@
 #include "kv_append.cuh"
 #include "lmhead.cuh"
 #include "mamba_scan.cuh"
+#include "spec_verify.cuh"
 #include "unmask.cuh"
 
 namespace {
@@ -111,6 +112,18 @@ bd_status bd_attn_step(const void *q, const void *k_prefix, const void *v_prefix
                        int H_q, int H_kv, int d, float scale, bd_dtype dtype, float *o,
                        float *lse, void *workspace, size_t workspace_bytes,
                        bd_stream_t stream) {
+  return bd_attn_step_ex(q, k_prefix, v_prefix, prefix_rows, k_blk, v_blk, prefix_len,
+                         prefix_offset, B, S, H_q, H_kv, d, scale, dtype, o, lse, workspace,
+                         workspace_bytes, 0, stream);
+}
+
+bd_status bd_attn_step_ex(const void *q, const void *k_prefix, const void *v_prefix,
+                          int64_t prefix_rows, const void *k_blk, const void *v_blk,
+                          const int32_t *prefix_len, const int64_t *prefix_offset, int B, int S,
+                          int H_q, int H_kv, int d, float scale, bd_dtype dtype, float *o,
+                          float *lse, void *workspace, size_t workspace_bytes, int flags,
+                          bd_stream_t stream) {
+  if (flags & ~BD_ATTN_BLOCK_CAUSAL) return BD_ERR_INVALID_ARG;
   bd_status st = attn_shape_ok(B, S, H_q, H_kv, d);
   if (st != BD_OK) return st;
   if (dtype != BD_DTYPE_F32 && dtype != BD_DTYPE_BF16) return BD_ERR_INVALID_ARG;
@@ -156,6 +169,7 @@ bd_status bd_attn_step(const void *q, const void *k_prefix, const void *v_prefix
   bd::attn_ws_layout(B, H_kv, M, d, G, &p.ws, static_cast<char *>(workspace));
   p.G = G;
   p.wait_ns = bd::kDefaultWaitNs;
+  p.block_causal = (flags & BD_ATTN_BLOCK_CAUSAL) ? 1 : 0;
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
 
   if (dtype == BD_DTYPE_BF16 && bd::tc_supported(p)) {
@@ -193,27 +207,15 @@ size_t bd_unmask_workspace_bytes(int rows, int V) {
   return bd::unmask_ws_layout(rows, unmask_grid(sms), nullptr, nullptr);
 }
 
-bd_status bd_unmask(const float *logits, const uint8_t *mask, float gamma, int32_t *tokens_out,
-                    float *conf_out, uint8_t *commit_out, uint8_t *mask_out, int rows, int V,
-                    int block_S, int commit_at_least_one, void *workspace,
-                    size_t workspace_bytes, bd_stream_t stream) {
-  if (rows < 0 || rows > bd::kUnmaskMaxRows || V < 1) return BD_ERR_INVALID_ARG;
-  if (block_S < 0 || block_S > bd::kUnmaskFinalizeRows) return BD_ERR_INVALID_ARG;
-  if (commit_at_least_one && block_S < 1) return BD_ERR_INVALID_ARG;
-  if (std::isnan(gamma)) return BD_ERR_INVALID_ARG;
-  if (rows == 0) return BD_OK;
-  if (!logits || !mask || !tokens_out || !conf_out || !commit_out || !workspace)
-    return BD_ERR_INVALID_ARG;
-  if (!aligned16(logits) || !aligned16(workspace) ||
-      (reinterpret_cast<uintptr_t>(tokens_out) & 3u) ||
-      (reinterpret_cast<uintptr_t>(conf_out) & 3u))
-    return BD_ERR_INVALID_ARG;
+// The two unmask kernels on validated arguments (mask == nullptr: every row).
+static bd_status unmask_launch(const float *logits, const uint8_t *mask, float gamma,
+                               int32_t *tokens_out, float *conf_out, uint8_t *commit_out,
+                               uint8_t *mask_out, int rows, int V, int block_S,
+                               int commit_at_least_one, void *workspace, bd_stream_t stream) {
   const int sms = sm_count();
   if (sms <= 0) return BD_ERR_CUDA;
   const int G = unmask_grid(sms);
   if (rows / G + 3 > bd::kUnmaskRowList) return BD_ERR_UNSUPPORTED;
-  if (workspace_bytes < bd::unmask_ws_layout(rows, G, nullptr, nullptr))
-    return BD_ERR_INVALID_ARG;
   cudaStream_t cs = reinterpret_cast<cudaStream_t>(stream);
 
   bd::UnmaskParams rp = {};
@@ -246,6 +248,29 @@ bd_status bd_unmask(const float *logits, const uint8_t *mask, float gamma, int32
   const int grid = (rows + fp.rows_per_cta - 1) / fp.rows_per_cta;
   launch_pdl(bd::unmask_finalize_kernel, dim3(grid), dim3(bd::kUnmaskFinalizeThreads), 0, cs, fp);
   return check_launch();
+}
+
+bd_status bd_unmask(const float *logits, const uint8_t *mask, float gamma, int32_t *tokens_out,
+                    float *conf_out, uint8_t *commit_out, uint8_t *mask_out, int rows, int V,
+                    int block_S, int commit_at_least_one, void *workspace,
+                    size_t workspace_bytes, bd_stream_t stream) {
+  if (rows < 0 || rows > bd::kUnmaskMaxRows || V < 1) return BD_ERR_INVALID_ARG;
+  if (block_S < 0 || block_S > bd::kUnmaskFinalizeRows) return BD_ERR_INVALID_ARG;
+  if (commit_at_least_one && block_S < 1) return BD_ERR_INVALID_ARG;
+  if (std::isnan(gamma)) return BD_ERR_INVALID_ARG;
+  if (rows == 0) return BD_OK;
+  if (!logits || !mask || !tokens_out || !conf_out || !commit_out || !workspace)
+    return BD_ERR_INVALID_ARG;
+  if (!aligned16(logits) || !aligned16(workspace) ||
+      (reinterpret_cast<uintptr_t>(tokens_out) & 3u) ||
+      (reinterpret_cast<uintptr_t>(conf_out) & 3u))
+    return BD_ERR_INVALID_ARG;
+  const int sms = sm_count();
+  if (sms <= 0) return BD_ERR_CUDA;
+  if (workspace_bytes < bd::unmask_ws_layout(rows, unmask_grid(sms), nullptr, nullptr))
+    return BD_ERR_INVALID_ARG;
+  return unmask_launch(logits, mask, gamma, tokens_out, conf_out, commit_out, mask_out, rows, V,
+                       block_S, commit_at_least_one, workspace, stream);
 }
 
 bd_status bd_kv_append(void *k_prefix, void *v_prefix, int64_t prefix_rows, const void *k_new,
@@ -451,6 +476,45 @@ bd_status bd_mamba_block_scan(const float *x, const float *dt, const float *B_fw
     return BD_ERR_CUDA;
   }
   kern<<<dim3(H, B), (P / rb) * (N / 32), smem, reinterpret_cast<cudaStream_t>(stream)>>>(p);
+  return check_launch();
+}
+
+size_t bd_spec_verify_workspace_bytes(int rows, int V) {
+  const size_t u = bd_unmask_workspace_bytes(rows, V);
+  if (u == 0) return 0;
+  return bd::align256(u) + bd::align256(size_t(rows));  // + the threshold commits, unused here
+}
+
+bd_status bd_spec_verify(const float *logits, const int32_t *draft, int32_t *tokens_out,
+                         float *conf_out, uint8_t *commit_out, int32_t *n_accept_out, int rows,
+                         int V, int S, void *workspace, size_t workspace_bytes,
+                         bd_stream_t stream) {
+  if (rows < 0 || rows > bd::kUnmaskMaxRows || V < 1 || S < 1 || S > bd::kVerifyThreads)
+    return BD_ERR_INVALID_ARG;
+  if (rows % S != 0) return BD_ERR_INVALID_ARG;
+  if (rows == 0) return BD_OK;
+  if (!logits || !draft || !tokens_out || !conf_out || !commit_out || !n_accept_out || !workspace)
+    return BD_ERR_INVALID_ARG;
+  if (!aligned16(logits) || !aligned16(workspace) || (reinterpret_cast<uintptr_t>(draft) & 3u) ||
+      (reinterpret_cast<uintptr_t>(n_accept_out) & 3u) ||
+      (reinterpret_cast<uintptr_t>(tokens_out) & 3u) || (reinterpret_cast<uintptr_t>(conf_out) & 3u))
+    return BD_ERR_INVALID_ARG;
+  const size_t u = bd_unmask_workspace_bytes(rows, V);
+  if (u == 0) return BD_ERR_CUDA;
+  if (workspace_bytes < bd_spec_verify_workspace_bytes(rows, V)) return BD_ERR_INVALID_ARG;
+  uint8_t *thr_commit = static_cast<uint8_t *>(workspace) + bd::align256(u);
+  // every row's argmax and confidence: the unmask kernels over all rows
+  bd_status st = unmask_launch(logits, nullptr, 0.5f, tokens_out, conf_out, thr_commit, nullptr,
+                               rows, V, 0, 0, workspace, stream);
+  if (st != BD_OK) return st;
+  bd::VerifyParams vp = {};
+  vp.ar_tokens = tokens_out;
+  vp.draft = draft;
+  vp.commit_out = commit_out;
+  vp.n_accept = n_accept_out;
+  vp.S = S;
+  bd::spec_verify_kernel<<<rows / S, bd::kVerifyThreads, 0,
+                           reinterpret_cast<cudaStream_t>(stream)>>>(vp);
   return check_launch();
 }
 

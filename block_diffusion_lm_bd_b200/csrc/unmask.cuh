@@ -59,6 +59,11 @@ __host__ __device__ inline size_t unmask_ws_layout(int rows, int G, UnmaskWs *ws
   return off;
 }
 
+// A null mask (library-internal callers only) takes every row.
+__device__ __forceinline__ bool um_masked(const uint8_t *mask, int r) {
+  return mask == nullptr || mask[r] != 0;
+}
+
 struct UnmaskParams {
   const float *logits;
   const uint8_t *mask;
@@ -171,7 +176,7 @@ __global__ void __launch_bounds__(kUnmaskThreads, kUnmaskCtasPerSm)
   const int chunk = (p.rows + kUnmaskThreads - 1) / kUnmaskThreads;
   const int r_lo = min(p.rows, tid * chunk), r_hi = min(p.rows, r_lo + chunk);
   int cnt = 0;
-  for (int r = r_lo; r < r_hi; ++r) cnt += (p.mask[r] != 0);
+  for (int r = r_lo; r < r_hi; ++r) cnt += um_masked(p.mask, r);
   int s_total;
   const int excl = block_excl_scan(cnt, s_warp, &s_total);
   const int n_masked = s_total;
@@ -186,7 +191,7 @@ __global__ void __launch_bounds__(kUnmaskThreads, kUnmaskCtasPerSm)
   {
     int rk = excl;
     for (int r = r_lo; r < r_hi; ++r) {
-      const bool mk = p.mask[r] != 0;
+      const bool mk = um_masked(p.mask, r);
       if (c == 0) p.ws.rank[r] = mk ? rk : -1;
       if (mk) {
         if (rk >= rho0 && rk <= rho1) s_rows[rk - rho0] = r;
@@ -321,7 +326,7 @@ __global__ void __launch_bounds__(kUnmaskFinalizeThreads)
   const int64_t W = int64_t(*p.ws.n_masked) * V;
   for (int lr = threadIdx.x; lr < p.rows_per_cta; lr += blockDim.x) {
     const int r = blockIdx.x * p.rows_per_cta + lr;
-    const uint8_t mk = (r < p.rows) ? (p.mask[r] != 0) : 0;
+    const uint8_t mk = (r < p.rows) ? um_masked(p.mask, r) : 0;
     s_mask[lr] = mk;
     s_commit[lr] = 0;
     s_conf[lr] = -1.0;

@@ -116,6 +116,25 @@ bd_status bd_attn_step(const void *q, const void *k_prefix, const void *v_prefix
                        float *lse, void *workspace, size_t workspace_bytes,
                        bd_stream_t stream);
 
+/* Flags of bd_attn_step_ex. */
+#define BD_ATTN_BLOCK_CAUSAL 1 /* block position i sees block keys 0 .. i only */
+
+/*
+ * bd_attn_step with options. flags = 0 is exactly bd_attn_step. With
+ * BD_ATTN_BLOCK_CAUSAL, block position i attends to every prefix key and to
+ * the block's keys 0 .. i only (causal inside the block): the verification
+ * pass of self-speculative decoding ("Nemotron-Labs Diffusion",
+ * self-speculation: the block drafted bidirectionally is checked causally).
+ * Other flag bits return BD_ERR_INVALID_ARG. Same arguments, limits and
+ * errors as bd_attn_step otherwise.
+ */
+bd_status bd_attn_step_ex(const void *q, const void *k_prefix, const void *v_prefix,
+                          int64_t prefix_rows, const void *k_blk, const void *v_blk,
+                          const int32_t *prefix_len, const int64_t *prefix_offset, int B, int S,
+                          int H_q, int H_kv, int d, float scale, bd_dtype dtype, float *o,
+                          float *lse, void *workspace, size_t workspace_bytes, int flags,
+                          bd_stream_t stream);
+
 /* ------------------------------------------------------------------------ */
 /* Confidence unmasking                                                     */
 /* ------------------------------------------------------------------------ */
@@ -228,6 +247,38 @@ bd_status bd_lmhead_unmask(const void *hidden, const void *w_vocab, const uint8_
                            uint8_t *mask_out, int rows, int V, int D, int block_S,
                            int commit_at_least_one, void *workspace, size_t workspace_bytes,
                            bd_stream_t stream);
+
+/* ------------------------------------------------------------------------ */
+/* Self-speculative verification                                            */
+/* ------------------------------------------------------------------------ */
+
+/* Workspace bytes of bd_spec_verify (0: invalid sizes or no usable device). */
+size_t bd_spec_verify_workspace_bytes(int rows, int V);
+
+/*
+ * Commit rule of self-speculative decoding ("Nemotron-Labs Diffusion",
+ * self-speculation: a block drafted bidirectionally is checked by a causal
+ * pass - bd_attn_step_ex with BD_ATTN_BLOCK_CAUSAL - and its matching prefix
+ * commits; at temperature 0 the result equals autoregressive decoding).
+ *
+ * rows = B * S positions, in blocks of S consecutive rows. Row i of block b
+ * holds the causal pass's prediction of block position i (the caller aligns
+ * the logits so). For every row: tokens_out = argmax (lowest id on ties),
+ * conf_out = its probability (as bd_unmask). For every block:
+ *   n_accept_out[b] = the number of leading positions with token == draft;
+ *   commit_out = 1 for positions 0 .. n-1 (draft confirmed) and for position n
+ *   when n < S (its tokens_out is the autoregressive token there); 0 after.
+ *
+ * Arguments (device pointers): logits float [rows, V] (16-byte aligned),
+ * draft int32 [rows], tokens_out int32 [rows], conf_out float [rows],
+ * commit_out uint8 [rows], n_accept_out int32 [rows / S], workspace >=
+ * bd_spec_verify_workspace_bytes(rows, V). Supported: 1 <= S <= 64,
+ * rows % S == 0, rows <= 65536. Launches three kernels.
+ */
+bd_status bd_spec_verify(const float *logits, const int32_t *draft, int32_t *tokens_out,
+                         float *conf_out, uint8_t *commit_out, int32_t *n_accept_out, int rows,
+                         int V, int S, void *workspace, size_t workspace_bytes,
+                         bd_stream_t stream);
 
 /* ------------------------------------------------------------------------ */
 /* Committing a finished block into the prefix cache                        */

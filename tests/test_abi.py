@@ -34,7 +34,8 @@ def test_header_declares_the_boundary():
     for required in ("bd_attn_step", "bd_attn_workspace_bytes", "bd_unmask",
                      "bd_unmask_workspace_bytes", "bd_get_device_status", "bd_status_string",
                      "bd_kv_append", "bd_lmhead_unmask", "bd_lmhead_unmask_workspace_bytes",
-                     "bd_mamba_block_scan"):
+                     "bd_mamba_block_scan", "bd_attn_step_ex", "bd_spec_verify",
+                     "bd_spec_verify_workspace_bytes"):
         assert required in names
 
 
@@ -251,3 +252,44 @@ def test_mamba_host_validation(lib, kw, code):
 
 def test_mamba_empty_batch_is_a_no_op(lib):
     assert _mamba(lib, B=0) == 0
+
+
+def test_attn_step_ex_rejects_unknown_flags(lib):
+    a = dict(q=16, kp=16, vp=16, rows=10, kb=16, vb=16, pl=16, po=16, B=2, S=16, Hq=8, Hkv=2, d=64,
+             scale=0.0, dtype=0, o=16, lse=0, ws=16, wsb=1 << 30)
+    vp = lambda x: ctypes.c_void_p(x) if x else None
+    st = lib.bd_attn_step_ex(vp(a["q"]), vp(a["kp"]), vp(a["vp"]), a["rows"], vp(a["kb"]),
+                             vp(a["vb"]), vp(a["pl"]), vp(a["po"]), a["B"], a["S"], a["Hq"],
+                             a["Hkv"], a["d"], a["scale"], a["dtype"], vp(a["o"]), vp(a["lse"]),
+                             vp(a["ws"]), a["wsb"], 6, None)
+    assert st == INVALID
+
+
+def _verify(lib, **kw):
+    a = dict(lg=16, dr=16, tok=16, conf=16, com=16, na=16, rows=32, V=100, S=16, ws=16,
+             wsb=1 << 30, st=0)
+    a.update(kw)
+    vp = lambda x: ctypes.c_void_p(x) if x else None
+    return lib.bd_spec_verify(vp(a["lg"]), vp(a["dr"]), vp(a["tok"]), vp(a["conf"]), vp(a["com"]),
+                              vp(a["na"]), a["rows"], a["V"], a["S"], vp(a["ws"]), a["wsb"],
+                              vp(a["st"]))
+
+
+@pytest.mark.parametrize("kw,code", [
+    (dict(S=0), INVALID),
+    (dict(S=65), INVALID),
+    (dict(rows=33), INVALID),          # not whole blocks
+    (dict(rows=-16), INVALID),
+    (dict(V=0), INVALID),
+    (dict(lg=0), INVALID),
+    (dict(dr=0), INVALID),
+    (dict(na=0), INVALID),
+    (dict(lg=20), INVALID),            # logits must be 16-byte aligned
+    (dict(dr=18), INVALID),
+])
+def test_spec_verify_host_validation(lib, kw, code):
+    assert _verify(lib, **kw) == code
+
+
+def test_spec_verify_zero_rows_is_a_no_op(lib):
+    assert _verify(lib, rows=0) == 0
