@@ -24,7 +24,8 @@ d=128, prefix 4096, block S=16, V=131072, gamma=0.9), synthetic data.
 * --workload 2 / 3: ragged S=32 prefixes / one 262144-token prefix; 4: the
   block loop (up to 16 steps of B=64 blocks, then the block commit into the
   prefix cache); 5: the LM head fused with unmasking (128 rows, D=4096,
-  V=131072); 6: one Mamba-2 layer's block-local bidirectional scan (B=64).
+  V=131072); 6: one Mamba-2 layer's block-local bidirectional scan (B=64);
+  7: the self-speculative verification step at the decode-step size.
 Under torchrun (N > 1) every rank runs an independent replica (replicas
 only: the step has no exchange); the time is the max over ranks.
 """
@@ -991,12 +992,205 @@ def run_mamba(args):
         dist.destroy_process_group()
 
 
+# --------------------------------------------------------------------------
+# self-speculative verification step (workload 7)
+# --------------------------------------------------------------------------
+def run_spec(args):
+    """The verification step of self-speculative decoding at the decode-step
+    size: the causal pass's attention (bd_attn_step_ex, causal inside the
+    block) and the commit rule over the pass's logits (bd_spec_verify) for B=8
+    drafted blocks of S=16. Drafts are the logits' argmax with each position
+    replaced by another token with probability 0.1 (drawn before timing). Four
+    rotating input sets, as in the decode-step bench."""
+    from block_diffusion_lm_bd_b200 import api, build as _build, workloads
+
+    world, rank, local = dist_env()
+    dev = torch.device("cuda", local)
+    torch.cuda.set_device(dev)
+    dist = init_dist(world, "nccl")
+    if rank == 0 and _build.needs_build():
+        _build.build()
+    barrier(dist, dev)
+    w = workloads.WORKLOADS[1]
+    nsets = args.sets
+    sets = make_sets(w, dev, nsets, rank)
+    B, S, H_q, H_kv, d, V = w.B, w.S, w.H_q, w.H_kv, w.d, w.V
+    rows = B * S
+    g = torch.Generator(device="cpu").manual_seed(w.seed(1000 * rank) + 7)
+    for inp in sets:
+        ar = inp["logits"].argmax(dim=1).to(torch.int32).cpu()
+        wrong = torch.rand(rows, generator=g) < 0.1
+        ar[wrong] = (ar[wrong] + 1) % V
+        inp["draft"] = ar.to(dev)
+    ws_a = torch.empty(api.attn_workspace_bytes(B, S, H_q, H_kv, d), dtype=torch.uint8, device=dev)
+    ws_v = torch.empty(int(api._lib().bd_spec_verify_workspace_bytes(rows, V)), dtype=torch.uint8,
+                       device=dev)
+    o = torch.empty((B, S, H_q, d), dtype=torch.float32, device=dev)
+    lse = torch.empty((B, H_q, S), dtype=torch.float32, device=dev)
+    outs = [dict(tok=torch.empty(rows, dtype=torch.int32, device=dev),
+                 conf=torch.empty(rows, dtype=torch.float32, device=dev),
+                 com=torch.empty(rows, dtype=torch.uint8, device=dev),
+                 n=torch.empty(B, dtype=torch.int32, device=dev)) for _ in range(nsets)]
+    stream = torch.cuda.Stream(device=dev)
+
+    def attn(i):
+        inp = sets[i % nsets]
+        api.attn_step(inp["q"], inp["k_prefix"], inp["v_prefix"], inp["k_blk"], inp["v_blk"],
+                      inp["prefix_len"], inp["prefix_offset"], o=o, lse=lse, workspace=ws_a,
+                      stream=stream, block_causal=True)
+
+    def step(i):
+        attn(i)
+        inp, out = sets[i % nsets], outs[i % nsets]
+        api.spec_verify(inp["logits"], inp["draft"], S, tokens_out=out["tok"], conf_out=out["conf"],
+                        commit_out=out["com"], n_accept_out=out["n"], workspace=ws_v, stream=stream)
+
+    def timed(fn, P, reps):
+        g_ = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_, stream=stream):
+            for i in range(P):
+                fn(i)
+        g_.replay()
+        torch.cuda.synchronize(dev)
+        a = torch.cuda.Event(enable_timing=True)
+        b = torch.cuda.Event(enable_timing=True)
+        with torch.cuda.stream(stream):
+            a.record(stream)
+            for _ in range(reps):
+                g_.replay()
+            b.record(stream)
+        torch.cuda.synchronize(dev)
+        return a.elapsed_time(b)
+
+    with torch.cuda.stream(stream):
+        for i in range(max(args.warmup, 3)):
+            step(i)
+    stream.synchronize()
+    assert api.get_device_status(stream) == 0
+    P = min(args.steps, 200)
+    reps = max(1, args.steps // P)
+    l0 = api.launch_count()
+    sampler = ClockSampler(dev)
+    with sampler:
+        barrier(dist, dev)
+        ms_local = timed(step, P, reps)
+        barrier(dist, dev)
+    launches = (api.launch_count() - l0) / P
+    value, ms = aggregate_throughput(rows * P * reps, ms_local, dist, dev)
+    attn_ms = max_over_ranks(timed(attn, P, reps), dist, dev) / (P * reps)
+    assert api.get_device_status(stream) == 0
+    n_acc = torch.stack([out["n"] for out in outs]).float()
+    committed = float((n_acc + (n_acc < S).float()).mean())
+    # e2e: q, block K/V, logits and drafts from pinned host memory, results back
+    keys_in = ["q", "k_blk", "v_blk", "logits", "draft"]
+    host = [{k: sets[s_][k].to("cpu").pin_memory() for k in keys_in} for s_ in range(nsets)]
+    res_host = [{k: torch.empty(outs[s_][k].shape, dtype=outs[s_][k].dtype).pin_memory()
+                 for k in ("tok", "com", "n")} for s_ in range(nsets)]
+    K = min(args.steps, args.e2e_steps)
+    a = torch.cuda.Event(enable_timing=True)
+    b = torch.cuda.Event(enable_timing=True)
+    with torch.cuda.stream(stream):
+        barrier(dist, dev)
+        a.record(stream)
+        for i in range(K):
+            s_ = i % nsets
+            for k in keys_in:
+                sets[s_][k].copy_(host[s_][k], non_blocking=True)
+            step(i)
+            for k in ("tok", "com", "n"):
+                res_host[s_][k].copy_(outs[s_][k], non_blocking=True)
+        b.record(stream)
+    torch.cuda.synchronize(dev)
+    e2e_ms = max_over_ranks(a.elapsed_time(b), dist, dev)
+    if rank == 0:
+        peak, peak_kind = hbm_peak()
+        lens = sets[0]["prefix_len_host"].tolist()
+        abytes, prefix_bytes = attn_bytes(w, lens)
+        achieved = abytes / (attn_ms * 1e6)
+        rec = {
+            "metric": "verification-step block-tokens/s (self-speculation)",
+            "value": value,
+            "unit": "block-tokens/s",
+            "n_gpus": world,
+            "steps": P * reps,
+            "warmup": args.warmup,
+            "ms_per_step": ms / (P * reps),
+            "higher_is_better": True,
+            "scaling": "weak",
+            "vs_baseline": None,
+            "dtype": "bf16",
+            "data": "synthetic (seeded; decode-step shapes; drafts = argmax with 10% of positions changed)",
+            "config": {"workload": "self-speculative verification: " + workload_label(w) +
+                                   ", causal inside the block, 4 rotating input sets (> L2)",
+                       "committed_per_block": committed,
+                       "parallelism": f"replicas x{world}"},
+            "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s",
+                         "frac": achieved / peak, "traffic": None, "peak_kind": peak_kind,
+                         "kernel": "bd_attn_step_ex (causal block) = attn_tc_kernel + combine",
+                         "algorithmic_bytes": abytes, "avg_call_us": attn_ms * 1e3},
+            "cpu_baseline": None,
+            "e2e": {"value": rows * K * world / (e2e_ms * 1e-3), "unit": "block-tokens/s",
+                    "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in host[0].values()),
+                    "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in res_host[0].values()),
+                    "steps": K, "ms_per_step": e2e_ms / K},
+            "gpu_launches": int(round(launches * P * reps)),
+            "clocks": sampler.summary(),
+        }
+        print(json.dumps(rec))
+    if dist is not None:
+        dist.destroy_process_group()
+
+
+def run_reference_spec(args, world):
+    """The oracle of the verification step on host cores: per unit, one KV-head
+    group of one decode-step sequence through the causal-in-block attention
+    and S/H_kv rows of the commit rule."""
+    from oracle.spec import causal_block_attention, verify_commit
+    from block_diffusion_lm_bd_b200 import workloads
+
+    w = workloads.WORKLOADS[1]
+    one, inp, logits, _ = oracle_unit_inputs(w, 0)
+    x = logits.numpy()
+    g = one.g
+    t, n, tokens = 0.0, 0, 0.0
+    budget = max(1.0, min(30.0, args.steps * 0.5))
+    while t < budget:
+        kv = n % one.H_kv
+        t0 = time.perf_counter()
+        causal_block_attention(inp["q"][:, :, kv * g:(kv + 1) * g], inp["k_prefix"][:, kv:kv + 1],
+                               inp["v_prefix"][:, kv:kv + 1], inp["k_blk"][:, :, kv:kv + 1],
+                               inp["v_blk"][:, :, kv:kv + 1], inp["prefix_len_host"],
+                               inp["prefix_offset_host"])
+        r = max(1, one.S // one.H_kv)
+        verify_commit(x[:r], np.argmax(x[:r], axis=1), r)
+        t += time.perf_counter() - t0
+        tokens += one.S / one.H_kv
+        n += 1
+    v = tokens / t
+    print(json.dumps({
+        "impl": "reference", "metric": "verification-step block-tokens/s (self-speculation)",
+        "value": v, "unit": "block-tokens/s", "n_gpus": world, "steps": n, "warmup": 0,
+        "ms_per_step": t / n * 1e3, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "f64", "data": "synthetic (seeded)",
+        "config": {"workload": "self-speculative verification: " + workload_label(w),
+                   "parallelism": "host cores"},
+        "cpu_baseline": {"value": v, "unit": "block-tokens/s", "cores": cpu_threads(),
+                         "kind": "oracle",
+                         "sample": f"{n} units in {t:.1f} s; one KV-head group of one sequence's "
+                                   "causal pass + its share of the commit rule per unit"},
+        "e2e": {"value": v, "unit": "block-tokens/s", "h2d_bytes_per_step": 0,
+                "d2h_bytes_per_step": 0}}))
+
+
 def run_reference(args):
     world, rank, _ = dist_env()
     if rank != 0:
         return
     from block_diffusion_lm_bd_b200 import workloads
 
+    if args.workload == 7:
+        run_reference_spec(args, world)
+        return
     w = workloads.WORKLOADS[args.workload]
     if args.workload == 6:
         v, n, t = mamba_cpu_sample(w, max(1.0, min(30.0, args.steps * 0.5)))
@@ -1066,7 +1260,7 @@ def main(argv=None):
     ap.add_argument("--steps", type=int, default=4000)
     ap.add_argument("--warmup", type=int, default=50)
     ap.add_argument("--impl", default="native", choices=["native", "reference"])
-    ap.add_argument("--workload", type=int, default=1, choices=[1, 2, 3, 4, 5, 6])
+    ap.add_argument("--workload", type=int, default=1, choices=[1, 2, 3, 4, 5, 6, 7])
     ap.add_argument("--graph-steps", type=int, default=400)
     ap.add_argument("--sets", type=int, default=4,
                     help="rotating input sets (4 keep every step's inputs out of L2)")
@@ -1084,6 +1278,8 @@ def main(argv=None):
         run_lmhead(args)
     elif args.workload == 6:
         run_mamba(args)
+    elif args.workload == 7:
+        run_spec(args)
     else:
         run_gpu(args)
 
