@@ -46,11 +46,11 @@ constexpr int kMambaMaxS = 64;
 
 constexpr float kMambaMinScale = 0x1p-30f;  // fold the decay product into u below this
 
-// shared floats: x, dt*x, dt_r*x [S][P]; per-chunk output partials [NC][S][P];
-// B and C of both directions [S][N]; per-step a, 1/a, a_r, 1/a_r and dt, dt_r [S]
+// shared floats: x [S][P]; per-chunk output partials [NC][S][P]; B and C of
+// both directions [S][N]; per-step a, 1/a, a_r, 1/a_r and dt, dt_r [S]
 __host__ __device__ inline size_t mamba_smem_bytes(int S, int P, int N) {
   const int NC = N / 32;
-  return sizeof(float) * (size_t(3 + NC) * S * P + size_t(4) * S * N + size_t(6) * S);
+  return sizeof(float) * (size_t(1 + NC) * S * P + size_t(4) * S * N + size_t(6) * S);
 }
 
 // The state is kept scaled: s[t] = pi[t] * u[t] with pi[t] the product of the
@@ -111,9 +111,7 @@ __global__ void __launch_bounds__(512, 1) mamba_scan_kernel(MambaParams p) {
   const int S = p.S, P = p.P, N = p.N, H = p.H, G = p.G;
   const int PR = P / RB;          // row slots per column chunk
   float *sx = sm;                 // x[t]            [S][P]
-  float *sxf = sx + S * P;        // dt[t] * x[t]    [S][P]
-  float *sxr = sxf + S * P;       // dt_r[t] * x[t]  [S][P]
-  float *syp = sxr + S * P;       // partials        [NC][S][P]
+  float *syp = sx + S * P;        // partials        [NC][S][P]
   float *sBf = syp + NC * S * P;  // [S][N] each
   float *sCf = sBf + S * N;
   float *sBr = sCf + S * N;
@@ -170,12 +168,6 @@ __global__ void __launch_bounds__(512, 1) mamba_scan_kernel(MambaParams p) {
   }
   asm volatile("cp.async.wait_all;" ::: "memory");
   __syncthreads();
-  for (int i = tid; i < S * P; i += nth) {
-    const int t = i / P;
-    sxf[i] = sdt[t] * sx[i];
-    sxr[i] = sdtr[t] * sx[i];
-  }
-  __syncthreads();
 
   float *yp = syp + c * S * P + q0;
   float w[RB], acc[RB];
@@ -193,7 +185,7 @@ __global__ void __launch_bounds__(512, 1) mamba_scan_kernel(MambaParams p) {
       ipi = 1.f;
     }
 #pragma unroll
-    for (int r = 0; r < RB; ++r) w[r] = sxf[t * P + q0 + r * PR] * ipi;
+    for (int r = 0; r < RB; ++r) w[r] = sdt[t] * sx[t * P + q0 + r * PR] * ipi;
     mamba_step<RB>(u, w, sBf + t * N + c * 32, sCf + t * N + c * 32, acc);
 #pragma unroll
     for (int r = 0; r < RB; ++r) yp[t * P + r * PR] = pi * acc[r];
@@ -217,7 +209,7 @@ __global__ void __launch_bounds__(512, 1) mamba_scan_kernel(MambaParams p) {
       ipi = 1.f;
     }
 #pragma unroll
-    for (int r = 0; r < RB; ++r) w[r] = sxr[t * P + q0 + r * PR] * ipi;
+    for (int r = 0; r < RB; ++r) w[r] = sdtr[t] * sx[t * P + q0 + r * PR] * ipi;
     mamba_step<RB>(u, w, sBr + t * N + c * 32, sCr + t * N + c * 32, acc);
 #pragma unroll
     for (int r = 0; r < RB; ++r) yp[t * P + r * PR] += pi * acc[r];

@@ -354,8 +354,8 @@ bd_status bd_kv_append(void *k_prefix, void *v_prefix, int64_t prefix_rows, cons
  *   y            [B, S, H, P]   output (must not overlap the inputs)
  * Supported: 1 <= S <= 64; P in {32, 64, 128}; N in {32, 64, 128};
  * H % G == 0; B <= 4096; and the block's inputs of one head must fit in
- * shared memory: 4 * ((3 + N/32) * S * P + 4 * S * N + 6 * S) <= 227 KiB
- * (S = 16 fits every P and N; S = 64 fits N <= 64). Otherwise BD_ERR_UNSUPPORTED / BD_ERR_INVALID_ARG and
+ * shared memory: 4 * ((1 + N/32) * S * P + 4 * S * N + 6 * S) <= 227 KiB
+ * (S = 16 fits every P and N; S = 64 fits N <= 64, and P <= 64 with N = 128). Otherwise BD_ERR_UNSUPPORTED / BD_ERR_INVALID_ARG and
  * nothing is launched. Arithmetic in float32 (expf for the decays).
  */
 bd_status bd_mamba_block_scan(const float *x, const float *dt, const float *B_fwd,

@@ -244,7 +244,7 @@ def _mamba(lib, **kw):
     (dict(y=0), INVALID),
     (dict(h0=20), INVALID),                      # h0 must be 16-byte aligned
     (dict(ptr=18), INVALID),
-    (dict(S=64, P=64, N=128), UNSUPPORTED),       # the block's inputs exceed shared memory
+    (dict(S=64, P=128, N=128), UNSUPPORTED),      # the block's inputs exceed shared memory
 ])
 def test_mamba_host_validation(lib, kw, code):
     assert _mamba(lib, **kw) == code

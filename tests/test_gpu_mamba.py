@@ -84,3 +84,11 @@ def test_strong_decay_does_not_overflow_the_scaled_state():
     assert torch.isfinite(y).all()
     ref = batch_block_scan(*[inp[k] for k in workloads.MAMBA_ARGS])
     assert _err(y, ref) <= TOL
+
+
+def test_longest_block_that_fits_shared_memory():
+    # S = 64 with P = 64, N = 128: the largest staged block of the bench's state shape
+    inp = workloads.mamba_inputs(W6, device=DEV, B=2, S=64, H=4, P=64, N=128, G=2)
+    y = _run(inp)
+    ref = batch_block_scan(*[inp[k] for k in workloads.MAMBA_ARGS])
+    assert _err(y, ref) <= TOL
