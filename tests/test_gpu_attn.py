@@ -234,3 +234,14 @@ def test_cuda_graph_replays_match_oracle():
         assert err <= ATTN_TOL[torch.bfloat16], (step, err, raw)
         assert float(np.abs(to_np(lse) - rl).max()) <= LSE_TOL[torch.bfloat16], step
     del g
+
+
+def test_more_sequences_than_threads_tensor_core_path():
+    # 1000 sequences > the 320 threads of a tensor-core CTA: the in-kernel plan
+    # scans the lengths in several passes
+    w = _w(torch.bfloat16, 1000, 16, 32, 8, 128)
+    g = torch.Generator().manual_seed(13)
+    lens = torch.randint(0, 300, (1000,), generator=g).tolist()
+    inp = workloads.attention_inputs(w, device=DEV, lens=lens)
+    err = _sampled_check(inp, torch.bfloat16, n=64, seed=13)
+    print(f"B=1000 tensor-core path: sampled err/std {err:.2e}")

@@ -76,6 +76,7 @@ def _check(h, W, mask, gamma, block_S=0, fallback=False, workspace=None, rows_se
     (1, 64, 1, 1.0, 2),                # one row, one token, one K chunk
     (300, 128, 20000, 0.7, 3),         # three m tiles
     (4096, 64, 512, 1.0, 4),           # the most rows one call takes (32 m tiles)
+    (64, 16384, 1000, 1.0, 5),         # the largest hidden size (256 K chunks)
 ])
 def test_small_cases_match_oracle(rows, D, V, frac, seed):
     h, W = workloads.lmhead_inputs(W5.with_(V=V), device=DEV, step=seed, rows=rows, D=D, V=V)
