@@ -21,11 +21,12 @@
 //    finished accumulator and fold it into the row's running record with the
 //    numerics of the unmask kernels (fp32 exponentials, fp64 sums, exact
 //    rescale, lowest index on ties) while the MMA fills the other buffer.
-//    Each thread keeps one record per m tile and writes them at the end.
-//  * lh_finalize_kernel - per masked row, merges the 2 * G records (one warp
-//    per row, every record load issued before the first merge; CTAs of 16
-//    rows, or of one fallback block), confidence = 1 / sum, commit = conf >
-//    gamma in fp64, the optional per-block fallback, and the outputs.
+//    Each thread keeps one record per m tile; at the end the two halves of a
+//    row are merged and one record per (row, CTA) is written.
+//  * lh_finalize_kernel - per masked row, merges the G records (one warp per
+//    row, every record load issued before the first merge; CTAs of 16 rows, or
+//    of one fallback block), confidence = 1 / sum, commit = conf > gamma in
+//    fp64, the optional per-block fallback, and the outputs.
 #pragma once
 
 #include "attn_tc.cuh"
@@ -44,9 +45,9 @@ constexpr int kLhMaxMTiles = kLhMaxRows / kLhTile;
 constexpr uint32_t kLhTmemCols = 256;             // two 128-column accumulators
 constexpr int kLhGatherThreads = 256;
 constexpr int kLhFinalizeRows = 256;     // rows per finalize CTA at most
-constexpr int kLhFinalizeThreads = 256;
-constexpr int kLhMaxSms = 256;           // records per row = 2 * G <= 2 * kLhMaxSms
-constexpr int kLhRecPerLane = 2 * kLhMaxSms / 32;
+constexpr int kLhFinalizeThreads = 512;  // one warp per row of a 16-row CTA
+constexpr int kLhMaxSms = 256;           // records per row = G <= kLhMaxSms
+constexpr int kLhRecPerLane = kLhMaxSms / 32;
 
 constexpr uint32_t kLhSmBar = kLhStages * kLhStageBytes;
 constexpr int kLhNumBars = 2 * kLhStages + 5;
@@ -58,7 +59,7 @@ struct LhWs {
   int *n_masked;         // [1]
   int *rank;             // [rows]      rank among masked rows, -1 if unmasked
   __nv_bfloat16 *a;      // [rows_cap, D] hidden states of the masked rows, by rank
-  UnmaskPart *rec;       // [rows_cap][G][2] per-row records of each CTA and column half
+  UnmaskPart *rec;       // [rows_cap][G] per-row records of each CTA
 };
 
 __host__ __device__ inline size_t lh_ws_layout(int rows, int D, int G, LhWs *ws, char *base) {
@@ -71,7 +72,7 @@ __host__ __device__ inline size_t lh_ws_layout(int rows, int D, int G, LhWs *ws,
   if (ws) ws->a = reinterpret_cast<__nv_bfloat16 *>(base + off);
   off = align256(off + sizeof(__nv_bfloat16) * rows_cap * size_t(D));
   if (ws) ws->rec = reinterpret_cast<UnmaskPart *>(base + off);
-  off = align256(off + sizeof(UnmaskPart) * size_t(G) * 2 * rows_cap);
+  off = align256(off + sizeof(UnmaskPart) * size_t(G) * rows_cap);
   return off;
 }
 
@@ -322,15 +323,24 @@ __global__ void __launch_bounds__(kLhThreads, 1)
       }
       rs[mt] = s;
     }
-    // one record per (CTA, column half, masked row); rows of m tiles this CTA
-    // never touched get the empty record, so the finalize merges blindly
+    // one record per (CTA, masked row): the warp holding the second half of a
+    // row's columns hands its record over through shared memory (the stage
+    // ring is idle now: the last accumulator wait above means every MMA, and
+    // so every load, of this CTA has completed). Rows of m tiles this CTA never
+    // touched get the empty record, so the finalize merges blindly.
+    UnmaskPart *xch = reinterpret_cast<UnmaskPart *>(smem);
     for (int k = 0; k < n_mt; ++k) {
-      const int rho = k * kLhTile + lrow;
       UnmaskPart rec;
       rec.m = rm[k];
       rec.idx = ri[k];
       rec.sum = rs[k];
-      p.ws.rec[int64_t(rho) * (2 * p.G) + cta * 2 + hf] = rec;
+      if (hf == 1) xch[lrow] = rec;
+      named_bar_sync(1, 256);
+      if (hf == 0) {
+        um_merge(rec, xch[lrow]);
+        p.ws.rec[int64_t(k * kLhTile + lrow) * p.G + cta] = rec;
+      }
+      named_bar_sync(1, 256);
     }
   }
 
@@ -359,7 +369,7 @@ __global__ void __launch_bounds__(kLhFinalizeThreads) lh_finalize_kernel(LhFinal
   __shared__ uint8_t s_commit[kLhFinalizeRows];
   __shared__ uint8_t s_mask[kLhFinalizeRows];
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
-  const int nparts = 2 * p.G;
+  const int nparts = p.G;
   pdl_wait_previous();
   for (int lr = warp; lr < p.rows_per_cta; lr += kLhFinalizeThreads / 32) {
     const int r = blockIdx.x * p.rows_per_cta + lr;
