@@ -365,8 +365,9 @@ bd_status bd_lmhead_unmask(const void *hidden, const void *w_vocab, const uint8_
 
   bd::EncodeTiledFn enc = bd::encode_tiled_fn();
   if (!enc) return BD_ERR_CUDA;
-  CUtensorMap ma, mw;
+  CUtensorMap ma, mh, mw;
   if (!bd::make_map_2d(enc, &ma, p.ws.a, uint64_t(D), uint64_t(p.rows_cap)) ||
+      !bd::make_map_2d(enc, &mh, hidden, uint64_t(D), uint64_t(rows)) ||
       !bd::make_map_2d(enc, &mw, w_vocab, uint64_t(D), uint64_t(V)))
     return BD_ERR_CUDA;
   static std::atomic<int> smem_set{-1};
@@ -398,7 +399,7 @@ bd_status bd_lmhead_unmask(const void *hidden, const void *w_vocab, const uint8_
     attr[0].val.programmaticStreamSerializationAllowed = 1;
     cfg.attrs = attr;
     cfg.numAttrs = 1;
-    cudaLaunchKernelEx(&cfg, bd::lh_gemm_kernel, ma, mw, p);
+    cudaLaunchKernelEx(&cfg, bd::lh_gemm_kernel, ma, mh, mw, p);
   }
   st = check_launch();
   if (st != BD_OK) return st;

@@ -10,7 +10,8 @@
 // Three kernels:
 //  * lh_gather_kernel - ranks of the masked rows (block scan of the mask in
 //    every CTA) and a copy of their hidden states into a dense bf16 tile
-//    [rows_cap, D] of the workspace, masked rank rho at row rho.
+//    [rows_cap, D] of the workspace, masked rank rho at row rho; skipped when
+//    every row is masked (the projection then reads the hidden states in place).
 //  * lh_gemm_kernel - one persistent CTA per SM over the items (n tile of
 //    128 tokens, m tile of 128 masked rows), ordered n-major so that the m
 //    tiles of one n tile run back to back and its 1 MB of W is read from HBM
@@ -122,6 +123,7 @@ __global__ void __launch_bounds__(kLhGatherThreads) lh_gather_kernel(LhParams p)
   }
   __syncthreads();
   const int n = s_total;
+  if (n == p.rows) return;  // every row masked: the projection reads the hidden states in place
   const int vec = p.D / 8;  // 16-byte vectors per row
   for (int rho = blockIdx.x; rho < n; rho += gridDim.x) {
     const int4 *src = reinterpret_cast<const int4 *>(p.hidden + int64_t(s_row[rho]) * p.D);
@@ -145,8 +147,8 @@ struct LhBars {
 };
 
 __global__ void __launch_bounds__(kLhThreads, 1)
-    lh_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_w,
-                   const LhParams p) {
+    lh_gemm_kernel(const __grid_constant__ CUtensorMap tm_a, const __grid_constant__ CUtensorMap tm_h,
+                   const __grid_constant__ CUtensorMap tm_w, const LhParams p) {
   extern __shared__ uint8_t smem_raw[];
   const uint32_t raw = smem_u32(smem_raw);
   const uint32_t sbase = (raw + 1023u) & ~1023u;
@@ -170,6 +172,7 @@ __global__ void __launch_bounds__(kLhThreads, 1)
     *abort_flag = 0;
     fence_barrier_init();
     prefetch_tmap(&tm_a);
+    prefetch_tmap(&tm_h);
     prefetch_tmap(&tm_w);
   }
   if (warp == 1) {
@@ -199,6 +202,9 @@ __global__ void __launch_bounds__(kLhThreads, 1)
     // nothing to project in this CTA's range (its records are still written)
   } else if (warp == 0) {
     if (lane == 0) {
+      // rows by rank: the gathered tile, or the hidden states themselves when
+      // every row is masked (rank = row)
+      const CUtensorMap *tma = (n_masked == p.rows) ? &tm_h : &tm_a;
       uint32_t t = 0;
       bool ok = true;
       for (int64_t it = e0; ok && it < e1; ++it) {
@@ -213,7 +219,7 @@ __global__ void __launch_bounds__(kLhThreads, 1)
           const uint32_t dst = sbase + st * kLhStageBytes;
           bar_expect_tx(bars.full + 8 * st, kLhStageBytes);
           const int kx = ((kc + k_rot) % nk) * kLhChunk;
-          tma_load_2d(dst, &tm_a, bars.full + 8 * st, kx, mt * kLhTile);
+          tma_load_2d(dst, tma, bars.full + 8 * st, kx, mt * kLhTile);
           tma_load_2d(dst + kLhPanel, &tm_w, bars.full + 8 * st, kx, nt * kLhTile);
         }
       }
