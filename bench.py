@@ -952,8 +952,31 @@ def run_mamba(args):
         except Exception:
             pass
         alu_peak = torch.cuda.get_device_properties(dev).multi_processor_count * 128 * 2 * sm_mhz * 1e6 / 1e12
-        flops = 8.0 * w.S * e["P"] * e["N"] * e["H"] * w.B  # both directions: update + output FMA
+        S_, P_, N_ = w.S, e["P"], e["N"]
+        if S_ <= 16:
+            # chunked form: h0 C, the B / B_r dot products of both triangles,
+            # M x; every input read once and y written once bound it (HBM)
+            kernel = "mamba_ssd_kernel"
+            flops = 2.0 * (S_ * P_ * N_ + S_ * (S_ + 1) * N_ + S_ * S_ * P_) * e["H"] * w.B
+        else:
+            kernel = "mamba_scan_kernel"
+            flops = 8.0 * S_ * P_ * N_ * e["H"] * w.B  # both directions: update + output FMA
         achieved = flops / (call_us * 1e-6) / 1e12
+        gbs = nbytes / (call_us * 1e3)
+        if kernel == "mamba_ssd_kernel":
+            roof = {"bound": "hbm", "achieved": gbs, "peak": peak, "unit": "GB/s",
+                    "frac": gbs / peak, "traffic": None, "peak_kind": peak_kind, "kernel": kernel,
+                    "algorithmic_bytes": nbytes, "avg_call_us": call_us,
+                    "algorithmic_flops": flops, "alu_tflops": achieved, "alu_peak": alu_peak,
+                    "alu_frac": achieved / alu_peak,
+                    "alu_peak_kind": "derived: SMs x 128 fp32 lanes x 2 x max SM clock"}
+        else:
+            roof = {"bound": "alu", "achieved": achieved, "peak": alu_peak,
+                    "unit": "TFLOP/s", "frac": achieved / alu_peak, "traffic": None,
+                    "peak_kind": "derived: SMs x 128 fp32 lanes x 2 x max SM clock",
+                    "kernel": kernel, "algorithmic_flops": flops,
+                    "avg_call_us": call_us, "hbm_bytes": nbytes,
+                    "hbm_gbs": gbs, "hbm_peak": peak, "hbm_peak_kind": peak_kind}
         rec = {
             "metric": "Mamba block scan block-tokens/s",
             "value": value,
@@ -972,13 +995,7 @@ def run_mamba(args):
                                    f"states {w.B * e['H'] * e['P'] * e['N'] * 4 >> 20} MiB "
                                    "(> L2), two rotating input sets",
                        "parallelism": f"replicas x{world}"},
-            "roofline": {"bound": "alu", "achieved": achieved, "peak": alu_peak,
-                         "unit": "TFLOP/s", "frac": achieved / alu_peak, "traffic": None,
-                         "peak_kind": "derived: SMs x 128 fp32 lanes x 2 x max SM clock",
-                         "kernel": "mamba_scan_kernel", "algorithmic_flops": flops,
-                         "avg_call_us": call_us, "hbm_bytes": nbytes,
-                         "hbm_gbs": nbytes / (call_us * 1e3), "hbm_peak": peak,
-                         "hbm_peak_kind": peak_kind},
+            "roofline": roof,
             "cpu_baseline": cpu,
             "e2e": {"value": tokens * K * world / (e2e_ms * 1e-3), "unit": "block-tokens/s",
                     "h2d_bytes_per_step": sum(t.numel() * 4 for t in host.values()),

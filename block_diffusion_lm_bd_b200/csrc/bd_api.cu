@@ -78,6 +78,35 @@ bd_status attn_shape_ok(int B, int S, int H_q, int H_kv, int d) {
 int attn_grid(int sms) { return sms; }
 int unmask_grid(int sms) { return sms * bd::kUnmaskCtasPerSm; }
 
+// Blocks of at most 16 tokens: the chunked kernel, one CTA per (head, sequence).
+template <int P, int N>
+bd_status mamba_ssd_launch_pn(const bd::MambaParams &p, cudaStream_t cs) {
+  using L = bd::SsdShape<P, N>;
+  if (L::kSmemBytes > 48 * 1024 &&
+      cudaFuncSetAttribute(bd::mamba_ssd_kernel<P, N>, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                           int(L::kSmemBytes)) != cudaSuccess) {
+    cudaGetLastError();
+    return BD_ERR_CUDA;
+  }
+  bd::mamba_ssd_kernel<P, N><<<dim3(p.H, p.B), L::kThreads, L::kSmemBytes, cs>>>(p);
+  return check_launch();
+}
+
+bd_status mamba_ssd_launch(const bd::MambaParams &p, cudaStream_t cs) {
+  switch (p.P * 1000 + p.N) {
+    case 32032: return mamba_ssd_launch_pn<32, 32>(p, cs);
+    case 32064: return mamba_ssd_launch_pn<32, 64>(p, cs);
+    case 32128: return mamba_ssd_launch_pn<32, 128>(p, cs);
+    case 64032: return mamba_ssd_launch_pn<64, 32>(p, cs);
+    case 64064: return mamba_ssd_launch_pn<64, 64>(p, cs);
+    case 64128: return mamba_ssd_launch_pn<64, 128>(p, cs);
+    case 128032: return mamba_ssd_launch_pn<128, 32>(p, cs);
+    case 128064: return mamba_ssd_launch_pn<128, 64>(p, cs);
+    case 128128: return mamba_ssd_launch_pn<128, 128>(p, cs);
+    default: return BD_ERR_UNSUPPORTED;
+  }
+}
+
 }  // namespace
 
 extern "C" {
@@ -461,6 +490,7 @@ bd_status bd_mamba_block_scan(const float *x, const float *dt, const float *B_fw
   p.P = P;
   p.N = N;
   p.G = G;
+  if (S <= bd::kSsdMaxS) return mamba_ssd_launch(p, reinterpret_cast<cudaStream_t>(stream));
   const size_t smem = bd::mamba_smem_bytes(S, P, N);
   if (smem > 227 * 1024) return BD_ERR_UNSUPPORTED;  // the block's inputs must fit on chip
   // two state rows per thread when that still leaves whole warps

@@ -353,10 +353,13 @@ bd_status bd_kv_append(void *k_prefix, void *v_prefix, int64_t prefix_rows, cons
  * copies them in 16-byte pieces); the other pointers 4-byte aligned.
  *   y            [B, S, H, P]   output (must not overlap the inputs)
  * Supported: 1 <= S <= 64; P in {32, 64, 128}; N in {32, 64, 128};
- * H % G == 0; B <= 4096; and the block's inputs of one head must fit in
- * shared memory: 4 * ((1 + N/32) * S * P + 4 * S * N + 6 * S) <= 227 KiB
- * (S = 16 fits every P and N; S = 64 fits N <= 64, and P <= 64 with N = 128). Otherwise BD_ERR_UNSUPPORTED / BD_ERR_INVALID_ARG and
- * nothing is launched. Arithmetic in float32 (expf for the decays).
+ * H % G == 0; B <= 4096. Blocks of at most 16 tokens are computed in the
+ * unrolled (chunked) form of the same recurrences and fit every P and N;
+ * longer blocks run the recurrence itself, whose inputs of one head must fit
+ * in shared memory: 4 * ((1 + N/32) * S * P + 4 * S * N + 6 * S) <= 227 KiB
+ * (S = 64 fits N <= 64, and P <= 64 with N = 128). Otherwise
+ * BD_ERR_UNSUPPORTED / BD_ERR_INVALID_ARG and nothing is launched.
+ * Arithmetic in float32 (expf for the decays).
  */
 bd_status bd_mamba_block_scan(const float *x, const float *dt, const float *B_fwd,
                               const float *C_fwd, const float *dt_rev, const float *B_rev,

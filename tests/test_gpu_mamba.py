@@ -38,6 +38,8 @@ def _err(y, ref):
     (1, 64, 2, 128, 64, 1),
     (5, 7, 16, 32, 128, 8),
     (2, 33, 6, 128, 128, 3),
+    (1, 16, 2, 128, 64, 1),    # chunked kernel, widest state rows
+    (2, 17, 4, 64, 128, 2),    # one token past the chunked kernel: the recurrence
 ])
 def test_small_cases_match_oracle(B, S, H, P, N, G):
     inp = workloads.mamba_inputs(W6, device=DEV, B=B, S=S, H=H, P=P, N=N, G=G)
@@ -73,10 +75,12 @@ def test_reverse_direction_sees_only_the_block():
     assert np.abs(d - dref).max() <= TOL * ref1.std()
 
 
-def test_strong_decay_does_not_overflow_the_scaled_state():
+@pytest.mark.parametrize("S", [16, 24])
+def test_strong_decay_does_not_overflow_the_scaled_state(S):
     # dt * |A| up to 60 per step: the decay product leaves the float32 range
-    # within two steps, so the kernel must fold it into the state
-    inp = workloads.mamba_inputs(W6, device=DEV, B=2, S=24, H=4, P=32, N=64, G=2)
+    # within two steps, so the recurrence must fold it into the state and the
+    # chunked form's decays underflow to zero without harm
+    inp = workloads.mamba_inputs(W6, device=DEV, B=2, S=S, H=4, P=32, N=64, G=2)
     inp["dt"] = inp["dt"] * 0 + torch.rand_like(inp["dt"]) * 4.0
     inp["dt_rev"] = inp["dt_rev"] * 0 + torch.rand_like(inp["dt_rev"]) * 4.0
     inp["A_fwd"] = inp["A_fwd"] * 0 - 15.0
@@ -90,5 +94,20 @@ def test_longest_block_that_fits_shared_memory():
     # S = 64 with P = 64, N = 128: the largest staged block of the bench's state shape
     inp = workloads.mamba_inputs(W6, device=DEV, B=2, S=64, H=4, P=64, N=128, G=2)
     y = _run(inp)
+    ref = batch_block_scan(*[inp[k] for k in workloads.MAMBA_ARGS])
+    assert _err(y, ref) <= TOL
+
+
+@pytest.mark.parametrize("S", [16, 20])
+def test_output_aligned_to_four_bytes_only(S):
+    inp = workloads.mamba_inputs(W6, device=DEV, B=2, S=S, H=4, P=64, N=64, G=2)
+    n = 2 * S * 4 * 64
+    buf = torch.full((n + 1,), float("nan"), device=DEV)
+    y = buf[1:].view(2, S, 4, 64)
+    assert y.data_ptr() % 16 == 4
+    api.mamba_block_scan(*[inp[k] for k in workloads.MAMBA_ARGS], y=y)
+    torch.cuda.synchronize()
+    assert api.get_device_status() == 0
+    assert torch.isnan(buf[:1]).all(), "nothing written before the output"
     ref = batch_block_scan(*[inp[k] for k in workloads.MAMBA_ARGS])
     assert _err(y, ref) <= TOL
