@@ -316,30 +316,23 @@ __global__ void __launch_bounds__(SsdShape<P, N>::kThreads, (P >= 128 ? 2 : 3))
   constexpr int NT = L::kThreads, N4 = N / 4, P4 = P / 4;
 
   // 1. Stage the operands with 16-byte asynchronous copies; rows of tokens
-  //    past the block are zero.
+  //    past the block are zero. The GEMM's right operand rows are h0 (P rows),
+  //    then B and B_r (16 rows each); C and C_r (16 rows each) follow them, so
+  //    all of it is one swizzled [P + 64][N] array.
   {
     const float4 z = make_float4(0.f, 0.f, 0.f, 0.f);
-    for (int q = tid; q < (L::kCols + 2 * kSsdMaxS) * N4; q += NT) {
-      const int r = q / N4, j = q % N4;
-      const float *src = nullptr;
-      float *dst;
-      if (r < P) {
-        src = p.h0 + ((int64_t(b) * H + h) * P + r) * N;
-        dst = sR + ssd_swz<N>(r, j);
-      } else if (r < L::kCols) {
-        const int s = (r - P) & (kSsdMaxS - 1);
-        if (s < S) src = (r < P + kSsdMaxS ? p.Bf : p.Br) + ((int64_t(b) * S + s) * G + g) * N;
-        dst = sR + ssd_swz<N>(r, j);
+    const float *h0b = p.h0 + (int64_t(b) * H + h) * (P * N);  // contiguous [P][N]
+#pragma unroll 4
+    for (int q = tid; q < P * N4; q += NT) cp_async16(sR + ssd_swz<N>(q / N4, q % N4), h0b + 4 * q);
+    for (int q = tid; q < 4 * kSsdMaxS * N4; q += NT) {
+      const int mat = q / (kSsdMaxS * N4), t = (q / N4) % kSsdMaxS, j = q % N4;
+      float *dst = sR + ssd_swz<N>(P + kSsdMaxS * mat + t, j);
+      if (t < S) {
+        const float *src = mat == 0 ? p.Bf : mat == 1 ? p.Br : mat == 2 ? p.Cf : p.Cr;
+        cp_async16(dst, src + ((int64_t(b) * S + t) * G + g) * N + 4 * j);
       } else {
-        const int t = (r - L::kCols) & (kSsdMaxS - 1);
-        const bool fw = r < L::kCols + kSsdMaxS;
-        if (t < S) src = (fw ? p.Cf : p.Cr) + ((int64_t(b) * S + t) * G + g) * N;
-        dst = (fw ? sCf : sCr) + ssd_swz<N>(t, j);
-      }
-      if (src)
-        cp_async16(dst, src + 4 * j);
-      else
         *reinterpret_cast<float4 *>(dst) = z;
+      }
     }
     for (int q = tid; q < kSsdMaxS * P4; q += NT) {
       const int t = q / P4, j = q % P4;
@@ -427,14 +420,14 @@ __global__ void __launch_bounds__(SsdShape<P, N>::kThreads, (P >= 128 ? 2 : 3))
   __syncthreads();
 
   // 4. y[t][p] = e^{F(0,t)} (h0 C[t])[p] + sum_s M[t][s] x[s][p] + D x[t][p];
-  //    thread tile 4 tokens x 4 channels.
+  //    thread tile 2 tokens x 4 channels.
   const float Dk = p.Dskip[h];
   const bool y16 = (reinterpret_cast<uintptr_t>(p.y) & 15u) == 0;
-  for (int q = tid; q < (kSsdMaxS / 4) * P4; q += NT) {
-    const int t0 = 4 * (q / P4), p0 = 4 * (q % P4);
-    float4 o[4];
+  for (int q = tid; q < (kSsdMaxS / 2) * P4; q += NT) {
+    const int t0 = 2 * (q / P4), p0 = 4 * (q % P4);
+    float4 o[2];
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < 2; ++i) {
       const float ef = sef[t0 + i];
       const float4 f = *reinterpret_cast<const float4 *>(sF + (t0 + i) * L::kFStride + p0);
       const float4 xv = *reinterpret_cast<const float4 *>(sX + (t0 + i) * P + p0);
@@ -445,7 +438,7 @@ __global__ void __launch_bounds__(SsdShape<P, N>::kThreads, (P >= 128 ? 2 : 3))
     for (int s = 0; s < kSsdMaxS; ++s) {
       const float4 xv = *reinterpret_cast<const float4 *>(sX + s * P + p0);
 #pragma unroll
-      for (int i = 0; i < 4; ++i) {
+      for (int i = 0; i < 2; ++i) {
         const float m = sM[(t0 + i) * kSsdMaxS + s];
         o[i].x = fmaf(m, xv.x, o[i].x);
         o[i].y = fmaf(m, xv.y, o[i].y);
@@ -454,7 +447,7 @@ __global__ void __launch_bounds__(SsdShape<P, N>::kThreads, (P >= 128 ? 2 : 3))
       }
     }
 #pragma unroll
-    for (int i = 0; i < 4; ++i) {
+    for (int i = 0; i < 2; ++i) {
       if (t0 + i >= S) continue;
       float *yo = p.y + ((int64_t(b) * S + t0 + i) * H + h) * P + p0;
       if (y16) {
