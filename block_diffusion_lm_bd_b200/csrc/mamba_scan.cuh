@@ -11,7 +11,10 @@
 //   y = y_fwd + y_rev.
 // The boundary state is read, never written.
 //
-// One CTA per (head, sequence); thread (c, q) owns state row q, columns
+// Two kernels compute it. Blocks of at most 16 tokens take mamba_ssd_kernel
+// (the unrolled, chunked form, further below). Longer blocks take
+// mamba_scan_kernel, the recurrence itself:
+// one CTA per (head, sequence); thread (c, q) owns state row q, columns
 // 32c .. 32c+31 of both directions in registers, a warp holding 32 rows of one
 // column chunk. The block's x, dt, B, C of the head's group are staged in
 // shared memory by asynchronous copies. A step is 32 FMAs of update and 32 of
